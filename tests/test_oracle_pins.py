@@ -1,0 +1,438 @@
+"""Pins of the oracle against facts fixed outside it: figures printed on the
+pages (tests/golden/page_figures.json), hand-derived encodings of the
+formats, library routines (torch's bf16 and float8_e4m3fn conversions and
+scaled_dot_product_attention), closed forms and brute force on tiny inputs.
+Each pin is chosen so that a plausible slip in the oracle (a wrong bit order,
+a dropped term, a transposed operand, an off-by-one page, a wrong GQA index)
+fails at least one of them.  CPU only."""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_bits(vals):
+    t = torch.tensor(np.asarray(vals, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- bf16 helpers
+
+def test_bf16_conversions_match_torch():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(20000).astype(np.float32) * np.float32(3.0)
+    # exact ties: low half 0x8000, both parities of the kept LSB
+    u = rng.integers(0, 2**31, 2000, dtype=np.uint64).astype(np.uint32)
+    ties = ((u & np.uint32(0x7F7F0000)) | np.uint32(0x8000)).view(np.float32)
+    x = np.concatenate([x, ties, -ties, np.float32([0.0, -0.0, 1e-40, -1e-40])])
+    ours = O.f32_to_bf16_rne(x)
+    ref = torch.tensor(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    back = O.bf16_to_f64(ref)
+    assert np.array_equal(back, torch.tensor(x).to(torch.bfloat16).double().numpy())
+
+
+# ------------------------------------------------------------------ packing
+
+def test_pack_literal_bytes():
+    # 00 -> 0, 01 -> +1, 11 -> -1, element i at bits 2*(i % 4) of byte i // 4
+    cases = {
+        (1, 0, 0, 0): 0x01, (-1, 0, 0, 0): 0x03, (0, 1, 0, 0): 0x04,
+        (0, 0, 0, -1): 0xC0, (-1, -1, -1, -1): 0xFF, (1, 1, 1, 1): 0x55,
+        (1, -1, 0, 1): 0x4D, (0, 0, 0, 0): 0x00, (0, 0, 1, 0): 0x10,
+    }
+    for codes, byte in cases.items():
+        assert O.pack_ternary(np.array(codes, np.int8))[0] == byte, codes
+
+
+def test_pack_roundtrip_exhaustive_and_no_field_10():
+    combos = np.array(list(itertools.product((-1, 0, 1), repeat=4)), dtype=np.int8)
+    assert len(combos) == 81
+    packed = O.pack_ternary(combos)                      # [81][1]
+    assert packed.shape == (81, 1)
+    assert len(set(packed[:, 0].tolist())) == 81          # injective
+    for b in packed[:, 0]:
+        for j in range(4):
+            assert (int(b) >> (2 * j)) & 3 != 0b10
+    assert np.array_equal(O.unpack_ternary(packed), combos)
+
+
+def test_unpack_rejects_field_10():
+    with pytest.raises(ValueError):
+        O.unpack_ternary(np.array([0x02], np.uint8))
+    with pytest.raises(ValueError):
+        O.pack_ternary(np.array([2, 0, 0, 0], np.int8))
+
+
+def test_group_element_order_row_major():
+    P, D = 16, 64
+    for (t, d) in [(0, 0), (0, 5), (3, 17), (15, 63)]:
+        x = np.zeros((1, 1, P, D), np.float32)
+        x[0, 0, t, d] = 1.0
+        codes, gamma = O.quantize_pack_ternary(bf16_bits(x))
+        flat = codes.reshape(-1)
+        i = t * D + d
+        nz = np.nonzero(flat)[0]
+        assert list(nz) == [i // 4]
+        assert flat[i // 4] == 1 << (2 * (i % 4))
+        assert gamma[0, 0] == np.float32(1.0 / (P * D))
+
+
+def test_storage_figures_vantage():
+    fig = json.load(open(os.path.join(GOLDEN, "page_figures.json")))
+    P = 16
+    for D in (64, 128, 256):
+        codes, _ = O.quantize_pack_ternary(bf16_bits(np.ones((1, 1, P, D))))
+        assert codes.nbytes * 8 / (P * D) == fig["ternary_bits_per_element"]["value"]
+    # one fp32 gamma per 16 x 256 group: 16 / 2.0078 -> 7.97x (as printed)
+    r = 16.0 / O.ternary_bits_per_element(P, 256)
+    assert round(r, fig["ternary_reduction_vs_fp16"]["decimals"]) == fig["ternary_reduction_vs_fp16"]["value"]
+    assert O.ternary_group_bytes(16, 128) == 516
+
+
+def test_storage_figures_minima():
+    fig = json.load(open(os.path.join(GOLDEN, "page_figures.json")))
+    f = fig["minima_bf16_kib_per_token"]
+    bf = O.kv_bytes_per_token(f["layers"], f["n_kv_heads"], f["head_dim"], 2)
+    f8 = O.kv_bytes_per_token(f["layers"], f["n_kv_heads"], f["head_dim"], 1)
+    assert bf == f["value"] * 1024
+    assert f8 == fig["minima_fp8_kib_per_token"]["value"] * 1024
+    g = fig["minima_gib_at_32k"]
+    assert bf * g["tokens"] / 2**30 == g["bf16"] and f8 * g["tokens"] / 2**30 == g["fp8"]
+    dep = fig["minima_deployed"]
+    assert round(bf / 1024 / dep["kib_per_token"], dep["decimals"]) == dep["reduction_vs_bf16"]
+    assert round(f8 / 1024 / dep["kib_per_token"], dep["decimals"]) == dep["reduction_vs_fp8"]
+    m = fig["minima_gib_per_million_tokens"]
+    assert round(bf * 1e6 / 2**30, m["decimals"]) == m["bf16"]
+    assert round(f8 * 1e6 / 2**30, m["decimals"]) == m["fp8"]
+    assert round(dep["kib_per_token"] * 1024 * 1e6 / 2**30, m["decimals"]) == m["deployed"]
+
+
+# ------------------------------------------------------------- gamma, codes
+
+def test_gamma_closed_forms():
+    rng = np.random.default_rng(1)
+    P, D = 16, 128
+    signs = rng.choice([-1.0, 1.0], size=(P, D))
+    assert O.ternary_gamma(O.bf16_to_f64(bf16_bits(0.375 * signs))) == np.float32(0.375)
+    two = np.where(rng.random((P, D)) < 0.5, 1.5, 0.25)
+    two[0, 0], two[0, 1] = 1.5, 0.25
+    k = (two == 1.5).sum()
+    expect = (1.5 * k + 0.25 * (P * D - k)) / (P * D)
+    assert O.ternary_gamma(two) == np.float32(expect)
+    assert O.ternary_gamma(np.zeros((P, D))) == 0.0
+    x = O.bf16_to_f64(bf16_bits(rng.standard_normal((P, D))))
+    assert O.ternary_gamma(4.0 * x) == 4.0 * O.ternary_gamma(x)          # exact scaling
+    assert O.ternary_gamma(x[::-1, ::-1]) == O.ternary_gamma(x)           # order-free
+
+
+def test_gamma_is_per_page_and_head():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((3, 2, 16, 64)).astype(np.float32)
+    x[:, 1] = 4.0 * x[:, 0]
+    x[2] *= 0.5
+    codes, gamma = O.quantize_pack_ternary(bf16_bits(x))
+    assert np.array_equal(gamma[:, 1], 4.0 * gamma[:, 0])
+    assert np.array_equal(codes[:, 1], codes[:, 0])
+    xb = O.bf16_to_f64(bf16_bits(x))
+    for p in range(3):
+        for h in range(2):
+            assert gamma[p, h] == np.float32(np.abs(xb[p, h]).mean())
+    # page selection and order
+    c2, g2 = O.quantize_pack_ternary(bf16_bits(x), page_ids=[2, 0])
+    assert np.array_equal(c2, codes[[2, 0]]) and np.array_equal(g2, gamma[[2, 0]])
+
+
+def test_codes_equal_literal_roundclip():
+    rng = np.random.default_rng(3)
+    for dist in ("normal", "laplace", "outlier"):
+        x = rng.standard_normal((16, 128))
+        if dist == "laplace":
+            x = rng.laplace(size=(16, 128))
+        if dist == "outlier":
+            x[:, :3] *= 10
+        x = O.bf16_to_f64(bf16_bits(x))
+        g = O.ternary_gamma(x)
+        c = O.ternary_codes(x, g)
+        literal = np.clip(np.round(x / float(g)), -1, 1)   # RoundClip, half-to-even
+        assert np.array_equal(c, literal.astype(np.int8))
+        assert set(np.unique(c).tolist()) <= {-1, 0, 1}
+
+
+def test_codes_at_threshold_ties():
+    # gamma = 1 exactly: half the group 1.5, half 0.5; threshold 0.5
+    P, D = 16, 64
+    x = np.full((P, D), 1.5)
+    x[:, D // 2:] = 0.5
+    x[0, 0], x[0, D // 2] = 1.49609375, 0.50390625   # sum unchanged; bf16 neighbours
+    x[1, 0], x[1, D // 2] = -1.5, -0.5
+    g = O.ternary_gamma(x)
+    assert g == np.float32(1.0)
+    c = O.ternary_codes(x, g)
+    assert c[0, D // 2] == 1          # just above the threshold
+    assert c[2, D // 2] == 0          # exactly at gamma / 2 -> tie -> 0
+    assert c[1, D // 2] == 0 and c[1, 0] == -1
+    assert c[2, 0] == 1
+
+
+def test_zero_group():
+    codes, gamma = O.quantize_pack_ternary(bf16_bits(np.zeros((1, 1, 16, 64))))
+    assert gamma[0, 0] == 0 and not codes.any()
+
+
+# ------------------------------------------------------------------- FP8
+
+def test_e4m3_known_codes():
+    # hand-derived from the OCP 8-bit floating point definition (E4M3: bias 7,
+    # max normal 448 = S.1111.110, min normal 2^-6, min subnormal 2^-9)
+    cases = [
+        (1.0, 0x38), (448.0, 0x7E), (-2.0, 0xC0), (0.5, 0x30), (2.0**-9, 0x01),
+        (2.0**-6, 0x08), (7 / 8 * 2.0**-6, 0x07), (1.125, 0x39),
+        (1.0625, 0x38),            # tie between 1.0 (even) and 1.125
+        (1.1875, 0x3A),            # tie between 1.125 and 1.25 (even)
+        (3 * 2.0**-10, 0x02),      # tie between 2^-9 and 2^-8 (even)
+        (2.0**-10, 0x00),          # tie between 0 (even) and 2^-9
+        (2.0**-10 * 1.0001, 0x01),
+        (-(2.0**-11), 0x80),       # negative underflow keeps its sign
+        (500.0, 0x7E), (-1e6, 0xFE), (464.0, 0x7E), (240.0, 0x77), (-0.0, 0x80),
+    ]
+    for v, code in cases:
+        got = O.f32_to_e4m3_rne_satfinite(np.float32([v]))[0]
+        assert got == code, (v, hex(got), hex(code))
+    assert np.array_equal(O.e4m3_to_f64(np.uint8([0x38, 0x7E, 0xC0, 0x01, 0x08])),
+                          [1.0, 448.0, -2.0, 2.0**-9, 2.0**-6])
+
+
+def test_e4m3_matches_torch_on_every_bf16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):          # the NaN bit patterns
+        x = O.bf16_to_f64(bits).astype(np.float32)
+    ok = np.isfinite(x) & (np.abs(x) <= 448.0)
+    ours = O.f32_to_e4m3_rne_satfinite(x[ok])
+    ref = torch.tensor(x[ok]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    big = np.isfinite(x) & (np.abs(x) > 448.0)
+    sat = O.f32_to_e4m3_rne_satfinite(x[big])
+    assert np.all((sat & 0x7F) == 0x7E)
+
+
+def test_e4m3_decode_matches_torch():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    ref = torch.tensor(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(O.e4m3_to_f64(codes), ref)
+    assert np.array_equal(O.f32_to_e4m3_rne_satfinite(O.e4m3_to_f64(codes).astype(np.float32)), codes)
+
+
+def test_fp8_page_scale():
+    x = np.zeros((1, 2, 16, 64), np.float32)
+    x[0, 0, 0, 0], x[0, 1, 5, 7] = 1.0, -8.0          # amax over all heads = 8
+    q, s = O.quantize_fp8_pages(bf16_bits(x))
+    assert s[0] == np.float32(8.0 / 448.0)
+    assert q[0, 1, 5, 7] == 0xFE                       # -8 * (448/8) = -448
+    assert q[0, 0, 0, 0] == O.f32_to_e4m3_rne_satfinite(np.float32([np.float32(1.0) * np.float32(448.0 / 8.0)]))[0]
+    q0, s0 = O.quantize_fp8_pages(bf16_bits(np.zeros((1, 1, 16, 64))))
+    assert s0[0] == 1.0 and not q0.any()
+
+
+# ------------------------------------------------------------- dequantise
+
+def test_dequantize_ternary_closed_form():
+    codes = O.pack_ternary(np.array([[1, 0, -1, 1] * 16] * 16, np.int8)).reshape(1, 1, 16, 16)
+    for g in (0.75, 1.0 / 3.0):
+        out = O.dequantize_ternary(codes, np.float32([[g]]))
+        row = np.array([g, 0.0, -g, g] * 16, np.float32)
+        assert np.array_equal(out[0, 0, 0], bf16_bits(row))
+
+
+def test_dequantize_fp8_closed_form():
+    e = np.zeros((1, 1, 16, 16), np.uint8)
+    e[0, 0, 0, :4] = [0x38, 0xC0, 0x7E, 0x01]          # 1, -2, 448, 2^-9
+    out = O.dequantize_fp8(e, np.float32([0.1]))
+    s = np.float32(0.1)
+    want = np.float32([s * np.float32(1), s * np.float32(-2), s * np.float32(448), s * np.float32(2.0**-9)])
+    assert np.array_equal(out[0, 0, 0, :4], bf16_bits(want))
+
+
+# -------------------------------------------------------------- attention
+
+def test_softmax_weights_sum_to_one_and_simple_cases():
+    rng = np.random.default_rng(4)
+    for L in (1, 7, 300):
+        q = rng.standard_normal(8)
+        k = rng.standard_normal((L, 8)) * 3
+        w = O.attention_full(q, k, np.eye(L), 0.5)        # V = I exposes the weights
+        assert abs(w.sum() - 1.0) < 1e-12 and (w >= 0).all()
+    v = rng.standard_normal((1, 8))
+    assert np.allclose(O.attention_full(rng.standard_normal(8), rng.standard_normal((1, 8)), v, 1.0), v[0], rtol=0, atol=1e-15)
+    vv = rng.standard_normal((50, 8))
+    kc = np.tile(rng.standard_normal(8), (50, 1))
+    assert np.allclose(O.attention_full(rng.standard_normal(8), kc, vv, 1.0), vv.mean(0), rtol=0, atol=1e-12)
+
+
+def test_attention_matches_sdpa():
+    rng = np.random.default_rng(5)
+    for L, D in ((5, 4), (333, 64), (1000, 256)):
+        q = rng.standard_normal(D)
+        k = rng.standard_normal((L, D))
+        v = rng.standard_normal((L, D))
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q)[None, None, None], torch.tensor(k)[None, None], torch.tensor(v)[None, None])
+        ours = O.attention_full(q, k, v, 1.0 / math.sqrt(D))
+        assert np.abs(ours - ref.numpy().reshape(-1)).max() < 1e-12
+
+
+def test_brute_force_tiny_long_double():
+    rng = np.random.default_rng(6)
+    for L in range(1, 9):
+        q = rng.standard_normal(4)
+        k = rng.standard_normal((L, 4))
+        v = rng.standard_normal((L, 4))
+        s = [np.longdouble(0.5) * sum(np.longdouble(q[d]) * np.longdouble(k[t, d]) for d in range(4)) for t in range(L)]
+        e = [np.exp(x) for x in s]
+        z = sum(e)
+        want = [sum(e[t] * np.longdouble(v[t, d]) for t in range(L)) / z for d in range(4)]
+        assert np.abs(O.attention_full(q, k, v, 0.5) - np.array(want, dtype=np.float64)).max() < 1e-13
+
+
+def test_split_merge_equals_full():
+    rng = np.random.default_rng(7)
+    L, D = 997, 32
+    q, k, v = rng.standard_normal(D), rng.standard_normal((L, D)) * 2, rng.standard_normal((L, D))
+    full = O.attention_full(q, k, v, 0.3)
+    for cuts in ([16], [1, 5, 400], [64 * i for i in range(1, 15)]):
+        edges = [0] + cuts + [L]
+        parts = [O.attention_partial(q, k[a:b], v[a:b], 0.3) for a, b in zip(edges, edges[1:])]
+        assert np.abs(O.merge_partials(parts) - full).max() < 1e-12
+        assert np.abs(O.merge_partials(parts[::-1]) - full).max() < 1e-12
+
+
+# ------------------------------------------------------- page classification
+
+def hp_pages(L, sink, window):
+    return [j for j in range(O.num_pages(L)) if O.page_format(j, L, sink, window, O.BF16, O.TERNARY) == O.BF16]
+
+
+def test_page_classification_hand_counts():
+    assert hp_pages(512, 4, 64) == [0, 28, 29, 30, 31]
+    assert hp_pages(4096, 4, 256) == [0] + list(range(240, 256))
+    assert len(hp_pages(32768, 4, 1024)) == 65
+    # ragged: L = 8200, window 2048 -> tokens 6152..8199 -> pages 384..512
+    assert hp_pages(8200, 4, 2048) == [0] + list(range(384, 513))
+    assert hp_pages(100, 0, 1) == [6]                  # only the (partial) last page
+    assert hp_pages(100, 17, 0) == [0, 1]              # sink spans two pages, no window
+    assert hp_pages(100, 0, 0) == []
+    assert hp_pages(100, 0, 500) == list(range(7))     # window longer than the context
+
+
+# ----------------------------------------------- decode over a hand-built cache
+
+def _hand_cache(D=16, hkv=2):
+    """Pools written directly from the encodings (no oracle quantiser): one
+    ternary page whose token rows are all +1 (0x55 bytes) or all -1 (0xFF),
+    one FP8 page of 1.0 (0x38) at scale s, one BF16 page of known values."""
+    P = 16
+    tern = np.zeros((1, hkv, P, D // 4), np.uint8)
+    for t in range(P):
+        tern[0, :, t, :] = 0x55 if t % 3 else 0xFF
+    gam = np.float32([[1.0 / 3.0, 0.75]])
+    fp8 = np.full((1, hkv, P, D), 0x38, np.uint8)
+    fp8[0, 1] = 0xC0                                    # -2.0 on KV head 1
+    s = np.float32([0.1])
+    rng = np.random.default_rng(8)
+    bfv = rng.standard_normal((1, hkv, P, D)).astype(np.float32)
+    bfb = bf16_bits(bfv)
+    cache = O.PagedCache(k_bf16=bfb, v_bf16=bfb[:, ::-1].copy(), k_fp8=fp8, v_fp8=fp8.copy(),
+                         k_fp8_scale=s, v_fp8_scale=np.float32([0.5]), k_tern=tern,
+                         v_tern=tern[:, :, ::-1].copy(), k_gamma=gam, v_gamma=gam[:, ::-1].copy())
+    # expected dense values, written from the encodings above
+    def dense(which, h):
+        t_rows = np.array([1.0 if t % 3 else -1.0 for t in range(P)])
+        if which == "v":
+            t_rows = t_rows[::-1]
+        g = float(gam[0, h]) if which == "k" else float(gam[0, ::-1][h])
+        tern_d = g * np.repeat(t_rows[:, None], D, axis=1)
+        f8v = (1.0 if h == 0 else -2.0) * float(s[0] if which == "k" else 0.5)
+        f8_d = np.full((P, D), f8v)
+        bf_d = O.bf16_to_f64(bfb[0, h] if which == "k" else bfb[0, ::-1][h])
+        return tern_d, f8_d, bf_d
+    return cache, dense
+
+
+@pytest.mark.parametrize("order", [(O.TERNARY, O.FP8_E4M3, O.BF16), (O.BF16, O.TERNARY, O.FP8_E4M3)])
+def test_decode_over_hand_built_cache_matches_sdpa(order):
+    D, hkv, G = 16, 2, 2
+    cache, dense = _hand_cache(D, hkv)
+    L = 16 * 3 - 5                                     # ragged last page
+    fmt = np.array([list(order) + [255]], np.uint8)
+    bt = np.zeros((1, 4), np.int32)
+    rng = np.random.default_rng(9)
+    qf = rng.standard_normal((1, hkv * G, D)).astype(np.float32)
+    qb = bf16_bits(qf)
+    out = O.decode_attention(qb, cache, bt, fmt, [L], hkv)
+    pos = {O.TERNARY: 0, O.FP8_E4M3: 1, O.BF16: 2}
+    for h in range(hkv * G):
+        g = h // G
+        ks, vs = [], []
+        for f in order:
+            ks.append(dense("k", g)[pos[f]])
+            vs.append(dense("v", g)[pos[f]])
+        k = torch.tensor(np.concatenate(ks)[:L])
+        v = torch.tensor(np.concatenate(vs)[:L])
+        qq = torch.tensor(O.bf16_to_f64(qb[0, h]))
+        ref = torch.nn.functional.scaled_dot_product_attention(qq[None, None, None], k[None, None], v[None, None])
+        assert np.abs(out[0, h] - ref.numpy().reshape(-1)).max() < 1e-12
+
+
+def test_decode_all_bf16_matches_sdpa_gqa_and_ignores_masked_slots():
+    rng = np.random.default_rng(10)
+    B, hq, hkv, D, L = 2, 6, 2, 32, 16 * 5 - 3
+    maxp = 5
+    k = rng.standard_normal((B, maxp, hkv, 16, D)).astype(np.float32)
+    v = rng.standard_normal((B, maxp, hkv, 16, D)).astype(np.float32)
+    q = rng.standard_normal((B, hq, D)).astype(np.float32)
+    lens = [L, 16 * 2 + 1]
+    kb, vb, qb = bf16_bits(k), bf16_bits(v), bf16_bits(q)
+    cache, bt, fmt = O.build_paged_cache(kb, vb, lens, sink=0, window=10**6, hp_fmt=O.BF16)
+    out = O.decode_attention(qb, cache, bt, fmt, lens, hkv)
+    for b in range(B):
+        Lb = lens[b]
+        kk = torch.tensor(O.bf16_to_f64(kb[b]).transpose(1, 0, 2, 3).reshape(hkv, -1, D)[:, :Lb])
+        vv = torch.tensor(O.bf16_to_f64(vb[b]).transpose(1, 0, 2, 3).reshape(hkv, -1, D)[:, :Lb])
+        kk = kk.repeat_interleave(hq // hkv, dim=0)    # HF repeat_kv grouping
+        vv = vv.repeat_interleave(hq // hkv, dim=0)
+        qq = torch.tensor(O.bf16_to_f64(qb[b]))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq[None], kk[None], vv[None])[0, :, 0]
+        assert np.abs(out[b] - ref.numpy()).max() < 1e-12
+    # garbage in the slots past each context length changes nothing
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 4, :, 13:] = 1e4
+    v2[0, 4, :, 13:] = -1e4
+    k2[1, 2, :, 1:] = 7e3
+    c2, bt2, f2 = O.build_paged_cache(bf16_bits(k2), bf16_bits(v2), lens, sink=0, window=10**6, hp_fmt=O.BF16)
+    assert np.array_equal(O.decode_attention(qb, c2, bt2, f2, lens, hkv), out)
+
+
+def test_physical_placement_is_invisible():
+    rng = np.random.default_rng(11)
+    B, hkv, D, maxp = 3, 2, 64, 12
+    k = bf16_bits(rng.standard_normal((B, maxp, hkv, 16, D)))
+    v = bf16_bits(rng.standard_normal((B, maxp, hkv, 16, D)))
+    q = bf16_bits(rng.standard_normal((B, 4, D)))
+    lens = [16 * 12, 16 * 9 + 4, 40]
+    older = np.where(rng.random((B, maxp)) < 0.3, O.BF16, O.TERNARY).astype(np.uint8)
+    c1, bt1, f1 = O.build_paged_cache(k, v, lens, 4, 20, O.FP8_E4M3, older_fmt=older)
+    c2, bt2, f2 = O.build_paged_cache(k, v, lens, 4, 20, O.FP8_E4M3, older_fmt=older, slot_key=rng.random((B, maxp)))
+    assert np.array_equal(f1, f2) and not np.array_equal(bt1, bt2)
+    o1 = O.decode_attention(q, c1, bt1, f1, lens, hkv)
+    o2 = O.decode_attention(q, c2, bt2, f2, lens, hkv)
+    assert np.abs(o1 - o2).max() < 1e-13
+    assert {O.BF16, O.FP8_E4M3, O.TERNARY} <= set(np.unique(f1).tolist())
