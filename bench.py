@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark: compress a batch's bf16 KV into the mixed-format paged cache and
+run one decode-attention pass over it (one "step"), on synthetic data shaped
+like the workload, through libkvc's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  The metric is HBM throughput: algorithmic
+bytes (what the method must read and write: bf16 source pages, packed codes
++ gamma, FP8 bytes + scales, BF16 pages, Q, block table, output) divided by
+device time.  `--impl reference` times the CPU oracle on a bounded sample
+of the same workload instead.  For N > 1 (torchrun) every rank runs its own
+independent batch (weak scaling, no collective on the data path).
+"""
+
+from __future__ import annotations
+
+import os
+
+os.environ.setdefault("OPENBLAS_NUM_THREADS", "1")   # the oracle baseline runs on one core
+os.environ.setdefault("OMP_NUM_THREADS", "1")
+
+import argparse
+import hashlib
+import json
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "decode-attention KV GB/s & % of B200 HBM peak; pack GB/s; oracle speedup"
+P = 16
+
+WORKLOAD_TEXT = {
+    "tiny": "tiny decode: B=1, Hq=8, Hkv=4, D=64, L=512, sink 4, window 64 BF16, older pages ternary",
+    "qwen3b": "Qwen2.5-3B-shaped layer: B=8, Hq=16, Hkv=2, D=128, L=4096, sink 4, window 256 FP8, older pages ternary, 2% outlier channels",
+    "llama8b": "Llama-3-8B-shaped layer: B=32, Hq=32, Hkv=8, D=128, L=32768, sink 4, window 1024 BF16, older pages ternary, random physical page placement",
+    "longctx": "long-context ragged layer: B=16, Hq=24, Hkv=4, D=256, L~U[8192,131072], sink 4, window 2048 FP8, 5% BF16 anchors, Laplace values",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+# ---------------------------------------------------------------- bytes
+
+def algorithmic_bytes(cfg, layout, B, max_pages, has_older):
+    """Bytes each kernel of one step must move, by kernel."""
+    H, D, hq = cfg["n_kv_heads"], cfg["head_dim"], cfg["n_q_heads"]
+    n_bf, n_f8, n_t = layout.pool_pages
+    page_bf16 = 2 * P * H * D
+    out = {
+        "pack_bf16": 2 * n_bf * (2 * page_bf16),
+        "pack_fp8": 2 * n_f8 * (page_bf16 + P * H * D + 4),
+        "pack_ternary": 2 * n_t * (page_bf16 + P * H * D // 4 + 4 * H),
+    }
+    total_pages = n_bf + n_f8 + n_t
+    out["decode"] = (2 * (n_bf * page_bf16 + n_f8 * (P * H * D + 4) + n_t * (P * H * D // 4 + 4 * H))
+                     + B * (2 * hq * D + 4 * hq * D + 4) + 4 * total_pages
+                     + (total_pages if has_older else 0))
+    return out
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].strip().lower() == "active"})
+        load = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------- our arm
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "compressed_decode_attention_kvc_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """dram bytes per launch recorded from an ncu capture of the current
+    kernel sources (profiles/ncu_traffic.txt), else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for line in open(path):
+        parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if parts.get("kernel") == kernel_key and parts.get("sources") == src and "bytes_per_launch" in parts:
+            return float(parts["bytes_per_launch"])
+    return None
+
+
+def run_ours(args, rank, world, dev, peak, peak_src):
+    import compressed_decode_attention_kvc_b200 as K
+    from compressed_decode_attention_kvc_b200 import paged_cache as PC
+
+    inp = synth.make_decode_inputs(args.workload, seed=rank, device=dev)
+    cfg = inp["cfg"]
+    B, max_pages, H, _, D = inp["k_pages"].shape
+    hq = cfg["n_q_heads"]
+    hp = K.KVC_FMT_BF16 if cfg["hp"] == "bf16" else K.KVC_FMT_FP8_E4M3
+    older = None
+    if inp["anchor"].any():
+        older = torch.where(inp["anchor"], K.KVC_FMT_BF16, K.KVC_FMT_TERNARY2).to(torch.uint8)
+    lens_h = inp["context_lens"].cpu()
+    sk = None if inp["slot_key"] is None else inp["slot_key"].cpu()
+    layout = PC.plan_paged_cache(lens_h, max_pages, cfg["sink"], cfg["window"], hp,
+                                 older_fmt=None if older is None else older.cpu(), slot_key=sk)
+    cache = PC.allocate_device_cache(layout, H, D, dev)
+    kf = inp["k_pages"].view(B * max_pages, H, P, D)
+    vf = inp["v_pages"].view(B * max_pages, H, P, D)
+    q, lens = inp["q"], inp["context_lens"]
+    ws_bytes = K.kvc_decode_workspace_size(B, hq, H, D, max_pages)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((B, hq, D), dtype=torch.float32, device=dev)
+    nbytes = algorithmic_bytes(cfg, layout, B, max_pages, older is not None)
+    stream = torch.cuda.current_stream()
+
+    pools = [(f, n) for f, n in zip((K.KVC_FMT_BF16, K.KVC_FMT_FP8_E4M3, K.KVC_FMT_TERNARY2),
+                                    layout.pool_pages) if n > 0]
+    names = {K.KVC_FMT_BF16: "pack_bf16", K.KVC_FMT_FP8_E4M3: "pack_fp8", K.KVC_FMT_TERNARY2: "pack_ternary"}
+    fields = {K.KVC_FMT_BF16: ("k_bf16", "v_bf16", None, None),
+              K.KVC_FMT_FP8_E4M3: ("k_fp8", "v_fp8", "k_fp8_scale", "v_fp8_scale"),
+              K.KVC_FMT_TERNARY2: ("k_tern", "v_tern", "k_gamma", "v_gamma")}
+    launches_per_step = 2 * len(pools) + 1
+
+    def step(ev=None):
+        marks = []
+        for f, n in pools:
+            kn, vn, ks, vs = fields[f]
+            pl = cache.pools
+            if ev is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            K.kvc_quantize_pack_pages(kf, cache.page_ids[f], n, P, H, D, f, pl[kn], pl[ks] if ks else None)
+            K.kvc_quantize_pack_pages(vf, cache.page_ids[f], n, P, H, D, f, pl[vn], pl[vs] if vs else None)
+            if ev is not None:
+                e1 = torch.cuda.Event(enable_timing=True)
+                e1.record(stream)
+                marks.append((names[f], e0, e1))
+        if ev is not None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        K.kvc_decode_attention_paged(q, cache.struct, cache.block_table, older, lens, B, hq, H, D, P,
+                                     max_pages, cfg["sink"], cfg["window"], hp, 0.0, out, ws, ws_bytes)
+        if ev is not None:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(stream)
+            marks.append(("decode", e0, e1))
+            ev.extend(marks)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])
+    clocks.start()
+    time.sleep(0.3)
+    marks = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(marks)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    per_kernel = {}
+    for name, e0, e1 in marks:
+        per_kernel.setdefault(name, []).append(e0.elapsed_time(e1))
+    flags = K.kvc_decode_read_error(ws, B, hq, H, D, max_pages)
+    if flags:
+        raise RuntimeError(f"device error flags {flags}")
+
+    step_bytes = sum(nbytes.values())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
+
+    kernels = {}
+    for name, ts in per_kernel.items():
+        avg = sum(ts) / len(ts)
+        gbs = nbytes[name] / (avg * 1e-3) / 1e9
+        kernels[name] = {"ms": round(avg, 5), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                         "bytes": int(nbytes[name]), "share": 0.0}
+    tot = sum(k["ms"] for k in kernels.values())
+    for k in kernels.values():
+        k["share"] = round(k["ms"] / tot, 4)
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+
+    def roof(name):
+        k = kernels[name]
+        traffic = ncu_traffic(name)
+        return {"bound": "hbm", "achieved": k["gbs"], "peak": peak, "unit": "GB/s",
+                "frac": k["frac"], "traffic": traffic, "kernel": name, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": k["bytes"]}
+
+    res = {
+        "value": value, "ms_per_step": ms_per_step, "kernels": kernels, "roofline": roof(dom),
+        "decode_roofline": roof("decode"), "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk, "step_bytes": step_bytes, "cfg": cfg,
+        "pages": {"bf16": layout.pool_pages[0], "fp8": layout.pool_pages[1], "ternary": layout.pool_pages[2]},
+    }
+
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out,
+                             step_bytes, world, dev, hp)
+    return res
+
+
+def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out, step_bytes,
+            world, dev, hp):
+    """Same step through the public API with host buffers: planner on the
+    host, H2D of the bf16 pages / Q / lengths / block table from pinned
+    memory, pack + decode, D2H of the output, all inside the timed region."""
+    B, max_pages, H, _, D = inp["k_pages"].shape
+    hq = cfg["n_q_heads"]
+    hk = torch.empty(kf.shape, dtype=kf.dtype, pin_memory=True)
+    hv = torch.empty(vf.shape, dtype=vf.dtype, pin_memory=True)
+    hk.copy_(kf)
+    hv.copy_(vf)
+    hq_t = inp["q"].cpu().pin_memory()
+    hl = inp["context_lens"].cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h_older = None if older is None else older.cpu()
+    sk = None if inp["slot_key"] is None else inp["slot_key"].cpu()
+    q_d = torch.empty_like(inp["q"])
+    l_d = torch.empty_like(inp["context_lens"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lay = PC.plan_paged_cache(hl, max_pages, cfg["sink"], cfg["window"], hp, older_fmt=h_older, slot_key=sk)
+        kf.copy_(hk, non_blocking=True)
+        vf.copy_(hv, non_blocking=True)
+        q_d.copy_(hq_t, non_blocking=True)
+        l_d.copy_(hl, non_blocking=True)
+        cache.block_table.copy_(lay.block_table.pin_memory(), non_blocking=True)
+        for f in range(3):
+            if lay.pool_pages[f]:
+                cache.page_ids[f].copy_(lay.pool_src_ids[f].pin_memory(), non_blocking=True)
+        PC.compress_into(cache, kf, vf)
+        K.kvc_decode_attention_paged(q_d, cache.struct, cache.block_table, older, l_d, B, hq, H, D, P,
+                                     max_pages, cfg["sink"], cfg["window"], hp, 0.0, out, ws, ws_bytes)
+        hout.copy_(out, non_blocking=True)
+        stream.synchronize()
+        return float(hout[0, 0, 0])
+
+    for _ in range(2):
+        step()
+    steps = max(2, min(args.steps, 10))
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = (hk.numel() * 2 + hv.numel() * 2 + hq_t.numel() * 2 + hl.numel() * 4
+           + layout.block_table.numel() * 4 + sum(len(x) for x in layout.pool_src_ids) * 4)
+    return {"value": step_bytes * world * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4),
+            "ms_per_step": ms / steps, "steps": steps}
+
+
+# --------------------------------------------------------- oracle arm
+
+def oracle_sample_step(inp, cfg, pairs):
+    """Oracle work on a bounded sample: compress every page of the sampled
+    (sequence, KV head) pairs and decode those pairs.  Returns algorithmic
+    bytes of the sample (same accounting as the GPU step)."""
+    import oracle as O
+    H, D = cfg["n_kv_heads"], cfg["head_dim"]
+    hq = cfg["n_q_heads"]
+    G = hq // H
+    nbytes = 0
+    for b, g in pairs:
+        L = int(inp["context_lens"][b])
+        kb = inp["k_pages"][b, :, g:g + 1].contiguous().view(torch.int16).numpy().view(np.uint16)
+        vb = inp["v_pages"][b, :, g:g + 1].contiguous().view(torch.int16).numpy().view(np.uint16)
+        hp = O.BF16 if cfg["hp"] == "bf16" else O.FP8_E4M3
+        older = None
+        if inp["anchor"].any():
+            older = np.where(inp["anchor"][b:b + 1].numpy(), O.BF16, O.TERNARY).astype(np.uint8)
+        cache, bt, fmt = O.build_paged_cache(kb[None], vb[None], [L], cfg["sink"], cfg["window"], hp,
+                                             older_fmt=older)
+        qb = inp["q"][b:b + 1, g * G:(g + 1) * G].contiguous().view(torch.int16).numpy().view(np.uint16)
+        O.decode_attention(qb, cache, bt, fmt, [L], 1)
+        n_bf, n_f8, n_t = cache.k_bf16.shape[0], cache.k_fp8.shape[0], cache.k_tern.shape[0]
+        grp = 2 * P * D
+        nbytes += 2 * n_bf * 2 * grp + 2 * n_f8 * (grp + P * D) + 2 * n_t * (grp + P * D // 4 + 4)
+        nbytes += 2 * (n_bf * grp + n_f8 * P * D + n_t * (P * D // 4 + 4)) + G * D * 6 + 4 * (n_bf + n_f8 + n_t)
+    return nbytes
+
+
+def oracle_inputs(workload):
+    """Two sequences of the workload (same shapes and value distributions
+    per sequence); the oracle arms sample (sequence, KV head) pairs from
+    them."""
+    return synth.make_decode_inputs(workload, seed=0, device="cpu", batch=2)
+
+
+def pick_pairs(cfg, inp, k, offset=0):
+    B, H = inp["q"].shape[0], cfg["n_kv_heads"]
+    return [((offset + i) % B, (offset + i) % H) for i in range(k)]
+
+
+def cpu_baseline(args, budget_s=12.0):
+    inp = oracle_inputs(args.workload)
+    cfg = inp["cfg"]
+    pairs_done, nbytes = 0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        nbytes += oracle_sample_step(inp, cfg, pick_pairs(cfg, inp, 1, pairs_done))
+        pairs_done += 1
+    dt = time.perf_counter() - t0
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{pairs_done} (sequence, KV head) pairs of the {args.workload} workload: oracle "
+                      f"pack of all their pages + fp64 decode attention, {dt:.1f} s on one host core"}
+
+
+def run_reference(args):
+    inp = oracle_inputs(args.workload)
+    cfg = inp["cfg"]
+    for i in range(args.warmup):
+        oracle_sample_step(inp, cfg, pick_pairs(cfg, inp, 1, i))
+    t0 = time.perf_counter()
+    nbytes = 0
+    for i in range(args.steps):
+        nbytes += oracle_sample_step(inp, cfg, pick_pairs(cfg, inp, 1, args.warmup + i))
+    dt = time.perf_counter() - t0
+    v = nbytes / dt / 1e9
+    sample = (f"each step: one (sequence, KV head) pair of the {args.workload} workload - oracle pack "
+              f"of all its pages + fp64 decode attention, on one host core")
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_block(args, cfg),
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def config_block(args, cfg):
+    ctx = cfg["context"]
+    return {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}",
+            "batch": cfg["batch"], "context": list(ctx) if isinstance(ctx, tuple) else ctx,
+            "n_q_heads": cfg["n_q_heads"], "n_kv_heads": cfg["n_kv_heads"], "head_dim": cfg["head_dim"],
+            "page_size": P, "step": "pack every page of the batch into its format (bf16 copy / fp8 / "
+                                    "ternary) + one decode-attention pass over the compressed cache",
+            "l2": "inputs larger than L2 (bf16 source pages of the batch exceed 126 MB)",
+            "parallelism": f"dp{args.gpus} (independent batch per GPU)"}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    peak, peak_src = load_peaks()
+    r = run_ours(args, rank, world, dev, peak, peak_src)
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(r["value"], 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": config_block(args, r["cfg"]),
+            "roofline": r["roofline"], "decode_roofline": r["decode_roofline"],
+            "kernels": r["kernels"], "pages": r["pages"], "gpu_launches": r["gpu_launches"],
+            "clocks": r["clocks"], "e2e": r.get("e2e"),
+        }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(args)
+            line["cpu_baseline"] = cb
+            line["oracle_speedup"] = round(line["value"] / cb["value"], 1)
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,74 @@
+// Internal declarations shared by the CUDA translation units of libkvc.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "kvc.h"
+
+namespace kvc {
+
+constexpr int kPage = KVC_PAGE_SIZE;   // tokens per page
+
+// Device error flags (bit mask written with atomicOr into the workspace).
+constexpr uint32_t kErrBlockTable = 1u;
+constexpr uint32_t kErrFormat = 2u;
+constexpr uint32_t kErrContext = 4u;
+constexpr uint32_t kErrTimeout = 8u;
+
+// Format of logical page j (length-L sequence): the high-precision format
+// if the page holds any of the first `sink` tokens or any of the last
+// `window` tokens, else the caller's tag for that older page.  Used by the
+// host planner and by the decode kernels, so both always agree.
+__host__ __device__ __forceinline__ int page_format(int j, int L, int sink, int window,
+                                                    int hp, int older) {
+  const int first = j * kPage;
+  const int last_valid = ((j + 1) * kPage < L ? (j + 1) * kPage : L) - 1;
+  return (first < sink || last_valid >= L - window) ? hp : older;
+}
+
+// ---------------------------------------------------------------- quantise
+cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, int n, int hkv, int d,
+                                 void* dst, float* gamma, cudaStream_t s);
+cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, int n, int hkv, int d,
+                             void* dst, float* scale, cudaStream_t s);
+cudaError_t launch_copy_pages(const void* src, const int32_t* page_ids, int n,
+                              size_t page_bytes, void* dst, cudaStream_t s);
+cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const int32_t* page_ids,
+                                   int n, int hkv, int d, void* dst, cudaStream_t s);
+cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids,
+                               int n, int hkv, int d, void* dst, cudaStream_t s);
+
+// ------------------------------------------------------------------ decode
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  kvc_paged_cache cache;
+  const int32_t* block_table;
+  const uint8_t* older_fmt;
+  const int32_t* ctx;
+  int B, Hq, Hkv, G, max_pages;
+  int sink, window, hp;
+  float scale_log2;          // softmax_scale * log2(e)
+  int n_splits, pages_per_split;
+  float* out;
+  uint32_t* err;             // device error word
+  uint32_t* tickets;         // [B][Hkv] merge tickets
+  float* partials;           // [B][Hkv][n_splits][G][D + 2]
+};
+
+struct DecodePlan {
+  int n_splits;
+  int pages_per_split;
+  size_t ticket_offset, partial_offset, bytes;
+};
+
+// Split-K plan and workspace layout for these shapes on the current device.
+cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, DecodePlan* plan);
+
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, cudaStream_t s);
+cudaError_t launch_decode_simple(const DecodeParams& p, int head_dim, cudaStream_t s);
+
+}  // namespace kvc

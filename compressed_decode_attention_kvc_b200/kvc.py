@@ -1,0 +1,186 @@
+"""ctypes binding of libkvc (include/kvc.h).
+
+Argument marshalling only: every function here has the name of the C entry
+point it calls, turns torch tensors into raw device or host pointers and the
+current CUDA stream into a cudaStream_t, and raises KvcError on a non-zero
+status.  All computation happens in the library's CUDA kernels; there is no
+Python or CPU fallback, and importing this module fails loudly when the
+library has not been built.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkvc.so")
+
+KVC_OK = 0
+KVC_ERR_INVALID_ARG = 1
+KVC_ERR_UNSUPPORTED = 2
+KVC_ERR_WORKSPACE = 3
+KVC_ERR_CUDA = 4
+KVC_ERR_DEVICE_CHECK = 5
+KVC_ERR_TIMEOUT = 6
+
+KVC_FMT_BF16 = 0
+KVC_FMT_FP8_E4M3 = 1
+KVC_FMT_TERNARY2 = 2
+
+PAGE_SIZE = 16
+
+# device error flags returned by kvc_decode_read_error
+ERR_BLOCK_TABLE = 1
+ERR_FORMAT = 2
+ERR_CONTEXT = 4
+ERR_TIMEOUT = 8
+
+EXPORTS = (
+    "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",
+    "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
+    "kvc_decode_read_error",
+)
+
+
+class KvcError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {_lib.kvc_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+class kvc_paged_cache(ctypes.Structure):
+    _fields_ = [
+        ("k_bf16", ctypes.c_void_p), ("v_bf16", ctypes.c_void_p),
+        ("k_fp8", ctypes.c_void_p), ("v_fp8", ctypes.c_void_p),
+        ("k_fp8_scale", ctypes.c_void_p), ("v_fp8_scale", ctypes.c_void_p),
+        ("k_tern", ctypes.c_void_p), ("v_tern", ctypes.c_void_p),
+        ("k_gamma", ctypes.c_void_p), ("v_gamma", ctypes.c_void_p),
+        ("n_pages", ctypes.c_int64 * 3),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m compressed_decode_attention_kvc_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int
+    lib.kvc_status_string.restype = ctypes.c_char_p
+    lib.kvc_status_string.argtypes = [st]
+    lib.kvc_quantize_pack_pages.restype = st
+    lib.kvc_quantize_pack_pages.argtypes = [vp, vp, i32, i32, i32, i32, st, vp, vp, vp]
+    lib.kvc_dequantize_pages.restype = st
+    lib.kvc_dequantize_pages.argtypes = [vp, vp, vp, i32, i32, i32, i32, st, vp, vp]
+    lib.kvc_plan_paged_cache.restype = st
+    lib.kvc_plan_paged_cache.argtypes = [vp, i32, i32, i32, i32, i32, st, vp, vp, vp, vp, vp, vp]
+    lib.kvc_decode_workspace_size.restype = st
+    lib.kvc_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kvc_decode_attention_paged.restype = st
+    lib.kvc_decode_attention_paged.argtypes = [
+        vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, i32, i32, i32, i32, i32, i32,
+        i32, i32, st, f32, vp, vp, ctypes.c_size_t, vp]
+    lib.kvc_decode_read_error.restype = st
+    lib.kvc_decode_read_error.argtypes = [vp, i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_uint32), vp]
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != KVC_OK:
+        raise KvcError(status, where)
+
+
+def kvc_status_string(status: int) -> str:
+    return _lib.kvc_status_string(status).decode()
+
+
+def kvc_quantize_pack_pages(src_bf16, page_ids, n, page_size, n_kv_heads, head_dim, mode,
+                            dst, dst_scale, stream=None) -> None:
+    _check(_lib.kvc_quantize_pack_pages(_ptr(src_bf16), _ptr(page_ids), n, page_size, n_kv_heads,
+                                        head_dim, mode, _ptr(dst), _ptr(dst_scale), _stream(stream)),
+           "kvc_quantize_pack_pages")
+
+
+def kvc_dequantize_pages(src, src_scale, page_ids, n, page_size, n_kv_heads, head_dim, mode,
+                         dst_bf16, stream=None) -> None:
+    _check(_lib.kvc_dequantize_pages(_ptr(src), _ptr(src_scale), _ptr(page_ids), n, page_size,
+                                     n_kv_heads, head_dim, mode, _ptr(dst_bf16), _stream(stream)),
+           "kvc_dequantize_pages")
+
+
+def kvc_plan_paged_cache(context_lens, batch, max_pages, page_size, sink_tokens, window_tokens,
+                         hp_mode, older_fmt, slot_key, block_table, page_fmt, pool_pages,
+                         pool_src_ids) -> None:
+    """All tensors are host (CPU) tensors: int32 / uint8 / float32 as in kvc.h."""
+    _check(_lib.kvc_plan_paged_cache(_ptr(context_lens), batch, max_pages, page_size, sink_tokens,
+                                     window_tokens, hp_mode, _ptr(older_fmt), _ptr(slot_key),
+                                     _ptr(block_table), _ptr(page_fmt), _ptr(pool_pages),
+                                     _ptr(pool_src_ids)),
+           "kvc_plan_paged_cache")
+
+
+def kvc_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, max_pages) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.kvc_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, max_pages,
+                                          ctypes.byref(out)),
+           "kvc_decode_workspace_size")
+    return out.value
+
+
+def make_paged_cache(k_bf16=None, v_bf16=None, k_fp8=None, v_fp8=None, k_fp8_scale=None,
+                     v_fp8_scale=None, k_tern=None, v_tern=None, k_gamma=None, v_gamma=None,
+                     n_pages=(0, 0, 0)) -> kvc_paged_cache:
+    c = kvc_paged_cache()
+    for name, t in (("k_bf16", k_bf16), ("v_bf16", v_bf16), ("k_fp8", k_fp8), ("v_fp8", v_fp8),
+                    ("k_fp8_scale", k_fp8_scale), ("v_fp8_scale", v_fp8_scale),
+                    ("k_tern", k_tern), ("v_tern", v_tern), ("k_gamma", k_gamma),
+                    ("v_gamma", v_gamma)):
+        setattr(c, name, _ptr(t))
+    for f in range(3):
+        c.n_pages[f] = int(n_pages[f])
+    return c
+
+
+def kvc_decode_attention_paged(q_bf16, cache: kvc_paged_cache, block_table, older_fmt,
+                               context_lens, batch, n_q_heads, n_kv_heads, head_dim, page_size,
+                               max_pages, sink_tokens, window_tokens, hp_mode, softmax_scale,
+                               out, workspace, workspace_bytes, stream=None) -> None:
+    _check(_lib.kvc_decode_attention_paged(
+        _ptr(q_bf16), ctypes.byref(cache), _ptr(block_table), _ptr(older_fmt), _ptr(context_lens),
+        batch, n_q_heads, n_kv_heads, head_dim, page_size, max_pages, sink_tokens, window_tokens,
+        hp_mode, float(softmax_scale), _ptr(out), _ptr(workspace), int(workspace_bytes),
+        _stream(stream)),
+        "kvc_decode_attention_paged")
+
+
+def kvc_decode_read_error(workspace, batch, n_q_heads, n_kv_heads, head_dim, max_pages,
+                          stream=None) -> int:
+    flags = ctypes.c_uint32(0)
+    _check(_lib.kvc_decode_read_error(_ptr(workspace), batch, n_q_heads, n_kv_heads, head_dim,
+                                      max_pages, ctypes.byref(flags), _stream(stream)),
+           "kvc_decode_read_error")
+    return flags.value

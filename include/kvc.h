@@ -1,0 +1,241 @@
+/*
+ * kvc.h - C ABI of libkvc: a compressed, mixed-format paged KV cache and
+ * single-token decode attention over it, for NVIDIA B200 (sm_100a).
+ *
+ * The cache layout follows two of the source pages:
+ *   - "Show HN: Vantage-V-AI" (newshot.cc), section "Core architecture":
+ *     keys and values quantised to ternary {-1, 0, +1} with an absmean scale
+ *     gamma = mean(|X|), packed 4 codes per uint8 byte (2.0 bit/element);
+ *     attention-sink tokens kept at full precision; section "Quick start":
+ *     the knobs max_active_tokens (recent window), sink_tokens and
+ *     quant_mode = "fp8" (dynamic FP8 streaming).
+ *   - "Minima-KV" (twodots.gr), sections "Recent, Anchor and Stale" and
+ *     "How mixed-format attention works": pages of one request held in
+ *     different formats (recent pages high precision, older anchor pages kept
+ *     at higher fidelity, stale pages compressed but still addressable), read
+ *     directly by format-specific code paths whose partial states (max
+ *     score, sum of exponentials, output) are merged by one online-softmax
+ *     normalisation.  Section "Why the KV cache becomes a bottleneck":
+ *     non-contiguous physical pages addressed through a block table.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must be CUDA device (or managed) memory on
+ *     the current device; "host" pointers are ordinary host memory.  The
+ *     caller owns every buffer; the library never allocates, frees or keeps
+ *     a pointer after the call returns.
+ *   - Calls that take a stream only enqueue work on it and never
+ *     synchronise; inputs must stay valid until that work completes.
+ *   - Argument errors are reported before anything is enqueued, as a
+ *     kvc_status; nothing is written in that case.
+ *   - Page size is fixed at 16 tokens; head_dim is 64, 128 or 256.
+ *
+ * Page layouts (HND: head-major inside each page; all little-endian):
+ *   BF16       [page][Hkv][16][D]    bf16
+ *   FP8_E4M3   [page][Hkv][16][D]    OCP e4m3 bytes; one float32 scale per
+ *                                    page (over all KV heads), value = s * e
+ *   TERNARY2   [page][Hkv][16][D/4]  2-bit codes, element i of a (page,
+ *                                    head) group's row-major [token][dim]
+ *                                    order in byte i/4 at bits 2*(i%4)..+1,
+ *                                    00 = 0, 01 = +1, 11 = -1 (10 unused,
+ *                                    read as 0); one float32 gamma per
+ *                                    (page, KV head), value = gamma * c
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVC_API __attribute__((visibility("default")))
+#else
+#define KVC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, passed through untouched (0 = the legacy default stream). */
+typedef struct CUstream_st* kvc_stream_t;
+
+typedef enum {
+  KVC_OK = 0,
+  KVC_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer, ... */
+  KVC_ERR_UNSUPPORTED = 2,   /* a shape this build does not handle (head_dim, page size, GQA > 8) */
+  KVC_ERR_WORKSPACE = 3,     /* workspace missing or smaller than kvc_decode_workspace_size() */
+  KVC_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  KVC_ERR_DEVICE_CHECK = 5,  /* a device-side check failed (see kvc_decode_read_error) */
+  KVC_ERR_TIMEOUT = 6        /* a device-side wait gave up after its iteration limit */
+} kvc_status;
+
+typedef enum {
+  KVC_FMT_BF16 = 0,
+  KVC_FMT_FP8_E4M3 = 1,
+  KVC_FMT_TERNARY2 = 2
+} kvc_format;
+
+#define KVC_PAGE_SIZE 16
+
+/* Human-readable name of a status code (static string, never NULL). */
+KVC_API const char* kvc_status_string(kvc_status status);
+
+/*
+ * kvc_quantize_pack_pages - compress whole pages into one page format.
+ *
+ * Ternary (Vantage, "Core architecture"; scale granularity per (page, KV
+ * head)): for each (page, KV head) group of 16*D values,
+ *   gamma = mean(|x|)  (float32, pairwise-tree sum),
+ *   code  = +1 if x > gamma/2, -1 if x < -gamma/2, else 0
+ *           (RoundClip(x / gamma, -1, +1), ties to 0),
+ * packed 4 per byte as described above; dst_scale receives gamma [n][Hkv].
+ * FP8 (Vantage "Quick start" quant_mode = "fp8"; Minima "Recent, Anchor and
+ * Stale", recent pages in FP8): per page, amax = max |x| over all heads,
+ *   s = amax / 448, e = round-to-nearest-even, saturating e4m3 of
+ *   x * (448 / amax) (float32 arithmetic); amax = 0 gives s = 1;
+ * dst_scale receives s [n].  BF16: dst[i] is a copy of the source page and
+ * dst_scale is ignored (may be NULL).
+ *
+ *   src_bf16   device, bf16 [n_src][Hkv][16][D]; 16-byte aligned
+ *   page_ids   device int32 [n]: dst page i is made from src page
+ *              page_ids[i]; NULL means page_ids[i] = i.  Entries must lie in
+ *              [0, n_src) (not checked on the device).
+ *   n          number of pages to produce (0 is a no-op)
+ *   page_size  must be 16
+ *   dst        device, layout of `mode` [n][...]; 16-byte aligned
+ *   dst_scale  device float32, [n][Hkv] (ternary) or [n] (FP8)
+ */
+KVC_API kvc_status kvc_quantize_pack_pages(const void* src_bf16, const int32_t* page_ids, int n,
+                                   int page_size, int n_kv_heads, int head_dim,
+                                   kvc_format mode, void* dst, float* dst_scale,
+                                   kvc_stream_t stream);
+
+/*
+ * kvc_dequantize_pages - expand compressed pages back to bf16 (the inverse
+ * used to re-expand a stale page; Minima, "Recent, Anchor and Stale").
+ * Ternary: bf16(gamma * c); FP8: bf16(s * e), the product in float32, both
+ * rounded to nearest even.  BF16: a copy.
+ *
+ *   src        device, layout of `mode`, [n_src][...]
+ *   src_scale  device float32: gamma [n_src][Hkv] (ternary) or s [n_src]
+ *              (FP8); ignored for BF16
+ *   page_ids   device int32 [n] or NULL: dst page i is made from src page
+ *              page_ids[i] (NULL: i)
+ *   dst_bf16   device bf16 [n][Hkv][16][D]; 16-byte aligned
+ */
+KVC_API kvc_status kvc_dequantize_pages(const void* src, const float* src_scale, const int32_t* page_ids,
+                                int n, int page_size, int n_kv_heads, int head_dim,
+                                kvc_format mode, void* dst_bf16, kvc_stream_t stream);
+
+/* Per-format page pools of one attention layer.  K and V are separate pools
+ * that share the block table: logical page j of sequence b lives in slot
+ * block_table[b][j] of the K and V pools of that page's format.  Pools of a
+ * format that no page uses may be NULL. */
+typedef struct kvc_paged_cache {
+  const void* k_bf16;          /* bf16 [n_pages[0]][Hkv][16][D] */
+  const void* v_bf16;
+  const void* k_fp8;           /* e4m3 [n_pages[1]][Hkv][16][D] */
+  const void* v_fp8;
+  const float* k_fp8_scale;    /* [n_pages[1]] */
+  const float* v_fp8_scale;
+  const void* k_tern;          /* packed [n_pages[2]][Hkv][16][D/4] */
+  const void* v_tern;
+  const float* k_gamma;        /* [n_pages[2]][Hkv] */
+  const float* v_gamma;
+  int64_t n_pages[3];          /* pool sizes, indexed by kvc_format */
+} kvc_paged_cache;
+
+/*
+ * kvc_plan_paged_cache - host-side page placement (a small block manager).
+ * Decides each logical page's format with the same rule the decode kernel
+ * applies, and gives every page a slot in the pool of its format.
+ *
+ * Format of logical page j of sequence b (length L = context_lens[b]):
+ *   hp_mode         if the page holds any of the first sink_tokens tokens
+ *                   or any of the last window_tokens tokens,
+ *   older_fmt[b][j] otherwise (TERNARY2 for stale pages, BF16 or FP8 for
+ *                   anchors; older_fmt == NULL means TERNARY2).
+ * Slots of each pool are handed out in increasing slot_key order (ties by
+ * logical index b*max_pages + j); slot_key == NULL gives logical order.
+ *
+ *   context_lens  host int32 [batch], each in [0, max_pages*16]
+ *   older_fmt     host uint8 [batch][max_pages] or NULL
+ *   slot_key      host float32 [batch][max_pages] or NULL
+ *   block_table   host int32 [batch][max_pages] out (unused entries 0)
+ *   page_fmt      host uint8 [batch][max_pages] out (unused entries 255)
+ *   pool_pages    host int32 [3] out: pages per format
+ *   pool_src_ids  host int32 [batch*max_pages] out: the logical page id
+ *                 b*max_pages + j held by each slot, format by format
+ *                 (BF16 slots first, then FP8, then ternary) - the page_ids
+ *                 to pass to kvc_quantize_pack_pages for each pool.
+ */
+KVC_API kvc_status kvc_plan_paged_cache(const int32_t* context_lens, int batch, int max_pages,
+                                int page_size, int sink_tokens, int window_tokens,
+                                kvc_format hp_mode, const uint8_t* older_fmt,
+                                const float* slot_key, int32_t* block_table,
+                                uint8_t* page_fmt, int32_t* pool_pages,
+                                int32_t* pool_src_ids);
+
+/*
+ * kvc_decode_workspace_size - bytes of device workspace that
+ * kvc_decode_attention_paged needs for these shapes on the current device
+ * (split-K partial states, merge tickets and an error word).
+ */
+KVC_API kvc_status kvc_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                     int max_pages, size_t* bytes);
+
+/*
+ * kvc_decode_attention_paged - one query token per sequence attends to its
+ * whole mixed-format paged cache (Minima, "How mixed-format attention
+ * works"; page formats as in kvc_plan_paged_cache).
+ *
+ * For query head h of sequence b (KV head g = h / (Hq/Hkv)):
+ *   s_t   = softmax_scale * q_h . k_hat_t        for t < L_b
+ *   out_h = sum_t softmax(s)_t * v_hat_t
+ * where k_hat, v_hat are the decoded cache values (bf16 value, s*e, or
+ * gamma*c, never re-rounded).  Each page is read in its own format; the
+ * sequence is split over pages, each split emits (max score, sum of
+ * exponentials, output) and the last split to finish merges them.  Tokens
+ * at or beyond L_b are masked; L_b = 0 gives a zero output row.
+ *
+ *   q_bf16        device bf16 [batch][Hq][D]
+ *   cache         host pointer to the pool descriptor (copied by value)
+ *   block_table   device int32 [batch][max_pages]
+ *   older_fmt     device uint8 [batch][max_pages] or NULL (all TERNARY2)
+ *   context_lens  device int32 [batch], each in [0, max_pages*16]
+ *   hp_mode       BF16 or FP8_E4M3: format of sink and window pages
+ *   softmax_scale <= 0 selects 1/sqrt(head_dim)
+ *   out           device float32 [batch][Hq][D]
+ *   workspace     device, >= kvc_decode_workspace_size() bytes, 256-byte
+ *                 aligned; its merge tickets must be zero before the first
+ *                 call (zero the whole buffer once); every call leaves them
+ *                 zero again, so one workspace serves repeated calls and
+ *                 CUDA-graph replay, but not two calls in flight at once.
+ * Device-side checks (block-table entry outside its pool, unknown page
+ * format, context length out of range) skip the offending page or
+ * sequence and set a flag that kvc_decode_read_error() returns.
+ */
+KVC_API kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache* cache,
+                                      const int32_t* block_table, const uint8_t* older_fmt,
+                                      const int32_t* context_lens, int batch, int n_q_heads,
+                                      int n_kv_heads, int head_dim, int page_size, int max_pages,
+                                      int sink_tokens, int window_tokens, kvc_format hp_mode,
+                                      float softmax_scale, float* out, void* workspace,
+                                      size_t workspace_bytes, kvc_stream_t stream);
+
+/*
+ * kvc_decode_read_error - synchronise `stream`, then read and clear the
+ * device error flags in `workspace` (as sized for these shapes).  *flags
+ * receives a bit mask: 1 = block-table entry out of range, 2 = unknown page
+ * format, 4 = context length out of range, 8 = a bounded wait timed out.
+ * Returns KVC_OK, or KVC_ERR_CUDA if the copy failed.
+ */
+KVC_API kvc_status kvc_decode_read_error(void* workspace, int batch, int n_q_heads, int n_kv_heads,
+                                 int head_dim, int max_pages, uint32_t* flags,
+                                 kvc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H */
