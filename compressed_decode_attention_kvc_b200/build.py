@@ -1,6 +1,6 @@
 """Build libkvc.so in this package directory with nvcc for sm_100a.
 
-    python -m compressed_decode_attention_kvc_b200.build [--force]
+    python compressed_decode_attention_kvc_b200/build.py [--force]
 
 Every .cu file under csrc/ is compiled into one shared library whose
 exported symbols are exactly the extern "C" entry points of include/kvc.h.

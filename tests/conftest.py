@@ -10,6 +10,14 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # build libkvc.so if it is missing or older than its sources (nvcc
+    # cross-compiles for sm_100a without a GPU)
+    import importlib.util
+    path = os.path.join(ROOT, "compressed_decode_attention_kvc_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_kvc_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
 
 
 @pytest.fixture(scope="session")
