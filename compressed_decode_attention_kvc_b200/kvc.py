@@ -41,8 +41,10 @@ ERR_TIMEOUT = 8
 EXPORTS = (
     "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
-    "kvc_decode_read_error",
+    "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc",
 )
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class KvcError(RuntimeError):
@@ -83,6 +85,10 @@ def _load() -> ctypes.CDLL:
     lib.kvc_decode_attention_paged.argtypes = [
         vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, i32, i32, i32, i32, i32, i32,
         i32, i32, st, f32, vp, vp, ctypes.c_size_t, vp]
+    lib.kvc_decode_attention_paged_noalloc.restype = st
+    lib.kvc_decode_attention_paged_noalloc.argtypes = [
+        vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, i32, i32, i32, i32, i32, i32,
+        i32, i32, st, f32, vp, vp]
     lib.kvc_decode_read_error.restype = st
     lib.kvc_decode_read_error.argtypes = [vp, i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_uint32), vp]
     return lib
@@ -184,3 +190,19 @@ def kvc_decode_read_error(workspace, batch, n_q_heads, n_kv_heads, head_dim, max
                                       max_pages, ctypes.byref(flags), _stream(stream)),
            "kvc_decode_read_error")
     return flags.value
+
+
+def kvc_decode_attention_paged_noalloc(q_bf16, cache: kvc_paged_cache, block_table, older_fmt,
+                                       context_lens, batch, n_q_heads, n_kv_heads, head_dim,
+                                       page_size, max_pages, sink_tokens, window_tokens, hp_mode,
+                                       softmax_scale, out, stream=None) -> None:
+    """kvc_decode_attention_paged without a caller-provided workspace: for
+    callers that cannot allocate device memory.  The library uses a fixed
+    device array of NOALLOC_SCRATCH_BYTES shared by every call on a device,
+    so calls that overlap on the GPU race; make the first call on each
+    device outside any stream capture."""
+    _check(_lib.kvc_decode_attention_paged_noalloc(
+        _ptr(q_bf16), ctypes.byref(cache), _ptr(block_table), _ptr(older_fmt), _ptr(context_lens),
+        batch, n_q_heads, n_kv_heads, head_dim, page_size, max_pages, sink_tokens, window_tokens,
+        hp_mode, float(softmax_scale), _ptr(out), _stream(stream)),
+        "kvc_decode_attention_paged_noalloc")

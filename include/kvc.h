@@ -234,6 +234,41 @@ KVC_API kvc_status kvc_decode_read_error(void* workspace, int batch, int n_q_hea
                                  int head_dim, int max_pages, uint32_t* flags,
                                  kvc_stream_t stream);
 
+/*
+ * kvc_decode_attention_paged_noalloc - kvc_decode_attention_paged for
+ * callers that cannot allocate device memory (code whose allocations all go
+ * through a framework's own pool, plugins with a fixed memory budget, or
+ * latency-critical paths that must not add a cudaMalloc).  The source
+ * pages have no counterpart of this entry point; it exists for such
+ * callers only.
+ *
+ * Same arguments and result as kvc_decode_attention_paged, without the
+ * workspace: the split-K partial states, merge tickets and error word live
+ * in a file-scope device array of KVC_NOALLOC_SCRATCH_BYTES bytes that
+ * every GPU loading the library holds until the process exits.  The call
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address on
+ *     that device (cudaGetSymbolAddress, with the device current) and caches
+ *     it; make that first call before any stream capture.
+ *   - Each call clears the error word and the merge tickets with
+ *     cudaMemsetAsync on `stream` before the kernel; the partial states are
+ *     fully rewritten.
+ *   - Every call on a device shares the one array: calls whose work
+ *     overlaps on the GPU (other streams, other host threads) race and give
+ *     wrong results.  Serialise them.
+ *   - Shapes whose workspace (kvc_decode_workspace_size) exceeds
+ *     KVC_NOALLOC_SCRATCH_BYTES are rejected with KVC_ERR_WORKSPACE.
+ *   - Device-side check flags are written into the shared array and are not
+ *     reported by this entry point.
+ */
+#define KVC_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+KVC_API kvc_status kvc_decode_attention_paged_noalloc(
+    const void* q_bf16, const kvc_paged_cache* cache, const int32_t* block_table,
+    const uint8_t* older_fmt, const int32_t* context_lens, int batch, int n_q_heads,
+    int n_kv_heads, int head_dim, int page_size, int max_pages, int sink_tokens,
+    int window_tokens, kvc_format hp_mode, float softmax_scale, float* out, kvc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
