@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -159,7 +161,7 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     import compressed_decode_attention_kvc_b200 as K
     from compressed_decode_attention_kvc_b200 import paged_cache as PC
 
-    inp = synth.make_decode_inputs(args.workload, seed=rank, device=dev)
+    inp = synth.make_decode_inputs(args.workload, seed=rank, device=dev, batch=args.batch)
     cfg = inp["cfg"]
     B, max_pages, H, _, D = inp["k_pages"].shape
     hq = cfg["n_q_heads"]

@@ -1,0 +1,838 @@
+// Mixed-format paged decode attention on the tensor cores (sm_100a).
+//
+// Method: "Minima-KV" (twodots.gr), section "How mixed-format attention
+// works" - every page is read in its own format directly as it is loaded (no
+// dense shadow copy), each split emits a partial state (max score, sum of
+// exponentials, output) and a common online-softmax normalisation merges
+// them.  Ternary pages follow "Show HN: Vantage-V-AI" (newshot.cc), section
+// "Core architecture" (codes {-1, 0, +1}, gamma = mean|X|, 4 codes per byte).
+//
+// Design (B200):
+// * Work: the (sequence, KV head, page) units of the whole batch are split
+//   evenly over every warp of a persistent grid ("stream-K"): warp W owns
+//   units [W*U/NW, (W+1)*U/NW), which may span several (sequence, KV head)
+//   pairs.  Each warp is an independent worker; no CTA-wide synchronisation
+//   after the prologue.  Ragged context lengths balance by construction.
+// * Staging: each warp keeps a 2-entry ring in shared memory; an entry holds
+//   up to 8 ternary pages, 2 FP8 pages or 1 BF16 page (K group then V group
+//   of one KV head), filled with 1-D TMA bulk copies (cp.async.bulk, no
+//   multicast) that complete on an mbarrier.  Page metadata (format, block-
+//   table slot, scales) for 32 units at a time is loaded lane-parallel one
+//   chunk ahead, so the warp never waits on a dependent global load.
+// * Math: mma.sync m16n8k16 (f16 in, f32 accumulate) with swapped operands:
+//   page tokens on M, the GQA group (<= 8 query heads) on N.  Q.K^T has the
+//   unpacked K page as A and Q as B; P.V has V^T as A and P^T as B (the
+//   score tile is transposed in registers with movmatrix).  Ternary codes are
+//   turned into f16 operands with one shift and one AND per pair of codes:
+//   the 2-bit field 01 / 11 placed at bits 14..15 of a half is +2.0 / -2.0
+//   exactly, 00 is 0.  FP8 pages convert with cvt.f16x2.e4m3x2, BF16 pages
+//   with a byte permute and cvt.f16x2.f32.  Tensor-core operands come from
+//   registers, so no unpacked copy of a page ever touches shared memory.
+// * Softmax: online, in log2 units, with a lazy maximum: the running maximum
+//   moves (and the accumulators are rescaled) only when a score exceeds it
+//   by more than 2^8, so P stays within f16 range without a cross-lane max
+//   on every page.  Per-page V scales are folded into P relative to a
+//   per-warp reference scale that is re-based when the ratio leaves
+//   [1/16, 16], keeping P far from the f16 subnormal range.
+// * Merge: each warp writes one partial state per (sequence, KV head) it
+//   touched; the last writer for a pair (an atomic ticket, no waiting)
+//   merges the pair's partials and writes the output rows.
+#include "kvc_internal.cuh"
+
+#include <math.h>
+
+namespace kvc {
+namespace {
+
+constexpr int kWarps = 4;            // warps per CTA; each is an independent worker
+constexpr int kEntries = 2;          // ring entries per warp
+constexpr int kMaxPages = 8;         // pages per entry (ternary)
+constexpr float kTau = 8.0f;         // lazy-max threshold, log2 units
+constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr int kSkip = 3;             // entry carrying an unusable page (flagged, no data)
+constexpr unsigned kFull = 0xffffffffu;
+
+struct Desc {
+  int fmt, np, bg, ntok_last;
+  float ks[kMaxPages], vs[kMaxPages];
+};
+
+template <int D>
+struct Shape {
+  static constexpr int kEntryBytes = 64 * D;   // one BF16 page: K group + V group
+  static constexpr int kHalf = 32 * D;         // K region | V region of an entry
+  static constexpr int kSteps = D / 16;        // k-steps of Q.K^T = m-tiles of P.V
+  static constexpr int kWPT = D / 64;          // K words (16 dims) per thread per token
+  static constexpr int kUPT = D / 64;          // V units (8 dims) per thread
+  static constexpr int kVW = kUPT > 1 ? kUPT / 2 : 1;   // V code words per thread per token
+};
+
+__host__ __device__ constexpr int group_bytes(int fmt, int d) {
+  return fmt == KVC_FMT_TERNARY2 ? 4 * d : (fmt == KVC_FMT_FP8_E4M3 ? 16 * d : 32 * d);
+}
+
+// ------------------------------------------------------------------ PTX
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait: false if the phase did not complete within the limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movtrans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  return __byte_perm(a, b, sel);
+}
+__device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Ternary fields at bit offset o (even, 0..14) of both 16-bit halves -> f16
+// pair of 2*code: 01 -> 0x4000 (+2), 11 -> 0xC000 (-2), 00 -> 0 (10 -> -0).
+__device__ __forceinline__ uint32_t tern2(uint32_t w, int o) {
+  return (o == 14 ? w : (w << (14 - o))) & 0xC000C000u;
+}
+// Two e4m3 bytes (low byte -> low half) -> f16x2.
+__device__ __forceinline__ uint32_t e4m3x2_f16(uint32_t two_bytes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xFFFFu), __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+// bf16x2 -> f16x2 (exact for |x| in the f16 normal range).
+__device__ __forceinline__ uint32_t bf16x2_f16(uint32_t u) {
+  return f16x2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+// byte-permute selector taking byte k and k+1 of a, interleaved with b's:
+// result bytes (a.k, b.k, a.k+1, b.k+1)
+__host__ __device__ constexpr uint32_t sel_pair(int k) {
+  return (uint32_t)(k | ((4 + k) << 4) | ((k + 1) << 8) | ((5 + k) << 12));
+}
+
+template <typename T>
+__device__ __forceinline__ T lds(const unsigned char* p) {
+  return *reinterpret_cast<const T*>(p);
+}
+
+// ------------------------------------------------------------- metadata
+struct Meta {          // one unit (page of one KV head), held by one lane
+  int fmt;             // page format, or kSkip when unusable
+  int phys;            // slot in the pool of that format
+  int bg;              // b * Hkv + g
+  int ntok;            // valid tokens of the page (1..16)
+  float ks, vs;        // K / V scale of the page (gamma, s, or 1)
+  int older;           // caller tag (phase A) before fmt is resolved
+  int j, L;            // page index, sequence length
+};
+
+struct Prologue {
+  const int* seqP;     // [B + 1] unit prefix over sequences
+  const int* seqL;     // [B] validated lengths
+};
+
+// Phase A: unit -> (sequence, KV head, page); block-table slot and caller tag.
+__device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prologue& pr, long long x,
+                                             long long u1, Meta& m) {
+  m.fmt = kSkip;
+  m.phys = -1;
+  m.bg = -1;
+  m.ntok = 0;
+  m.ks = m.vs = 0.f;
+  m.older = KVC_FMT_TERNARY2;
+  m.j = 0;
+  m.L = 0;
+  if (x >= u1) return;
+  int lo = 0, hi = p.B;          // seqP[lo] <= x < seqP[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pr.seqP[mid] <= x) lo = mid; else hi = mid;
+  }
+  const int b = lo;
+  const int L = pr.seqL[b];
+  const int np = (L + kPage - 1) / kPage;
+  const int off = (int)(x - pr.seqP[b]);
+  const int g = off / np;
+  const int j = off - g * np;
+  const long long row = (long long)b * p.max_pages + j;
+  m.bg = b * p.Hkv + g;
+  m.j = j;
+  m.L = L;
+  m.ntok = min(kPage, L - j * kPage);
+  m.phys = __ldg(p.block_table + row);
+  m.older = p.older_fmt ? (int)__ldg(p.older_fmt + row) : KVC_FMT_TERNARY2;
+}
+
+// Phase B: resolve the format, check the slot, load the scales.
+__device__ __forceinline__ void meta_phase_b(const DecodeParams& p, Meta& m) {
+  if (m.bg < 0) return;
+  const int fmt = page_format(m.j, m.L, p.sink, p.window, p.hp, m.older);
+  if (fmt < 0 || fmt > 2) {
+    atomicOr(p.err, kErrFormat);
+    m.fmt = kSkip;
+    return;
+  }
+  if (m.phys < 0 || m.phys >= p.cache.n_pages[fmt]) {
+    atomicOr(p.err, kErrBlockTable);
+    m.fmt = kSkip;
+    return;
+  }
+  m.fmt = fmt;
+  const int g = m.bg % p.Hkv;
+  if (fmt == KVC_FMT_TERNARY2) {
+    m.ks = __ldg(p.cache.k_gamma + (long long)m.phys * p.Hkv + g);
+    m.vs = __ldg(p.cache.v_gamma + (long long)m.phys * p.Hkv + g);
+  } else if (fmt == KVC_FMT_FP8_E4M3) {
+    m.ks = __ldg(p.cache.k_fp8_scale + m.phys);
+    m.vs = __ldg(p.cache.v_fp8_scale + m.phys);
+  } else {
+    m.ks = m.vs = 1.f;
+  }
+}
+
+// ----------------------------------------------------------- the worker
+template <int D>
+struct Worker {
+  using S = Shape<D>;
+  const DecodeParams& p;
+  const Prologue pr;
+  unsigned char* ring;     // this warp's kEntries entries
+  Desc* desc;              // [kEntries]
+  uint64_t* bars;          // [kEntries]
+  int lane, gid, tig;
+  long long u0, u1, cursor, cb;   // unit range, next unit to issue, chunk base
+  Meta cur, nxt;
+  bool nxt_b_pending;
+  int W, nwg;
+  long long U;
+  bool timed_out;
+
+  // per (sequence, KV head) state
+  int cur_bg;
+  uint32_t qf[2 * S::kSteps];
+  float acc[S::kSteps][4];
+  float m0, m1, l0, l1, uref;
+
+  __device__ Worker(const DecodeParams& pp, Prologue prr, unsigned char* r, Desc* d, uint64_t* b)
+      : p(pp), pr(prr), ring(r), desc(d), bars(b) {}
+
+  __device__ __forceinline__ int shfl(int v, int src) { return __shfl_sync(kFull, v, src); }
+
+  // Fill ring slot `slot` with the next entry.  Returns false when the
+  // warp's units are exhausted.
+  __device__ bool issue(int slot) {
+    if (cursor >= u1) return false;
+    int li = (int)(cursor - cb);
+    if (li >= 32) {
+      if (nxt_b_pending) meta_phase_b(p, nxt);
+      cur = nxt;
+      cb += 32;
+      li -= 32;
+      meta_phase_a(p, pr, cb + 32 + lane, u1, nxt);
+      nxt_b_pending = true;
+    } else if (nxt_b_pending) {
+      meta_phase_b(p, nxt);
+      nxt_b_pending = false;
+    }
+    const int f0 = shfl(cur.fmt, li);
+    const int bg0 = shfl(cur.bg, li);
+    int np = 1;
+    if (f0 != kSkip) {
+      const int cap = f0 == KVC_FMT_TERNARY2 ? kMaxPages : (f0 == KVC_FMT_FP8_E4M3 ? 2 : 1);
+      const bool ok = lane >= li && (cb + lane) < u1 && cur.fmt == f0 && cur.bg == bg0;
+      const uint32_t run = __ballot_sync(kFull, ok) >> li;
+      const int len = (run == 0xffffffffu) ? 32 : __ffs(~run) - 1;
+      np = min(len, cap);
+    }
+    const int ntok_last = shfl(cur.ntok, min(li + np - 1, 31));
+    Desc& d = desc[slot];
+    if (lane == li) {
+      d.fmt = f0;
+      d.np = np;
+      d.bg = bg0;
+      d.ntok_last = ntok_last;
+    }
+    if (lane >= li && lane < li + np) {
+      d.ks[lane - li] = cur.ks;
+      d.vs[lane - li] = cur.vs;
+    }
+    __syncwarp();
+    fence_proxy_async();
+    if (f0 == kSkip) {
+      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], 0);
+    } else {
+      const int gb = group_bytes(f0, D);
+      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(2 * np * gb));
+      __syncwarp();
+      if (lane >= li && lane < li + np) {
+        const int k = lane - li;
+        const int g = cur.bg % p.Hkv;
+        const long long grp = (long long)cur.phys * p.Hkv + g;
+        const unsigned char* ksrc;
+        const unsigned char* vsrc;
+        if (f0 == KVC_FMT_TERNARY2) {
+          ksrc = static_cast<const unsigned char*>(p.cache.k_tern);
+          vsrc = static_cast<const unsigned char*>(p.cache.v_tern);
+        } else if (f0 == KVC_FMT_FP8_E4M3) {
+          ksrc = static_cast<const unsigned char*>(p.cache.k_fp8);
+          vsrc = static_cast<const unsigned char*>(p.cache.v_fp8);
+        } else {
+          ksrc = static_cast<const unsigned char*>(p.cache.k_bf16);
+          vsrc = static_cast<const unsigned char*>(p.cache.v_bf16);
+        }
+        unsigned char* e = ring + slot * S::kEntryBytes;
+        bulk_g2s(e + k * gb, ksrc + grp * gb, (uint32_t)gb, &bars[slot]);
+        bulk_g2s(e + S::kHalf + k * gb, vsrc + grp * gb, (uint32_t)gb, &bars[slot]);
+      }
+    }
+    __syncwarp();
+    cursor += np;
+    return true;
+  }
+
+  __device__ __forceinline__ int warp_of(long long x) const {
+    return (int)(((x + 1) * (long long)nwg + U - 1) / U) - 1;
+  }
+
+  // Start a new (sequence, KV head): load Q as f16 B fragments, reset state.
+  __device__ void begin(int bg) {
+    cur_bg = bg;
+    const int b = bg / p.Hkv, g = bg - (bg / p.Hkv) * p.Hkv;
+    const int r = gid;                       // query head within the group
+    uint32_t raw[S::kWPT * 8];               // 16 * kWPT bf16 of row r
+    if (r < p.G) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint16_t*>(p.q) + ((long long)b * p.Hq + g * p.G + r) * D + 16 * tig * S::kWPT);
+#pragma unroll
+      for (int i = 0; i < 2 * S::kWPT; ++i) {
+        const uint4 v = __ldg(src + i);
+        raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < S::kWPT * 8; ++i) raw[i] = 0u;
+    }
+    // qf[ri] = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) + (ri & 7) (local dims)
+#pragma unroll
+    for (int ri = 0; ri < 2 * S::kSteps; ++ri) {
+      const int wl = ri >> 3, j = ri & 7;
+      const uint32_t wa = raw[8 * wl + (j >> 1)], wb = raw[8 * wl + 4 + (j >> 1)];
+      qf[ri] = bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
+    }
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[mt][c] = 0.f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+    uref = 0.f;
+  }
+
+  // Write this warp's partial state for cur_bg; the last writer merges.
+  __device__ void finish() {
+    if (cur_bg < 0) return;
+    const int bg = cur_bg;
+    const int G = p.G;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(kFull, l0, o);
+      l1 += __shfl_xor_sync(kFull, l1, o);
+    }
+    const int rs = G * (D + 2);
+    float* rec = p.partials + (long long)(W + bg) * rs;
+    const int c0 = 2 * tig, c1 = 2 * tig + 1;
+    if (gid == 0) {
+      if (c0 < G) { rec[c0 * (D + 2)] = m0; rec[c0 * (D + 2) + 1] = l0; }
+      if (c1 < G) { rec[c1 * (D + 2)] = m1; rec[c1 * (D + 2) + 1] = l1; }
+    }
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt) {
+      const int la = mt, lb = mt + S::kSteps;
+      const int da = 8 * (gid * S::kUPT + (la >> 3)) + (la & 7);
+      const int db = 8 * (gid * S::kUPT + (lb >> 3)) + (lb & 7);
+      if (c0 < G) {
+        rec[c0 * (D + 2) + 2 + da] = acc[mt][0] * uref;
+        rec[c0 * (D + 2) + 2 + db] = acc[mt][2] * uref;
+      }
+      if (c1 < G) {
+        rec[c1 * (D + 2) + 2 + da] = acc[mt][1] * uref;
+        rec[c1 * (D + 2) + 2 + db] = acc[mt][3] * uref;
+      }
+    }
+    __threadfence();
+    __syncwarp();
+    const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+    const int np = (pr.seqL[b] + kPage - 1) / kPage;
+    const long long sbg = pr.seqP[b] + (long long)g * np;
+    const int w_first = warp_of(sbg), w_last = warp_of(sbg + np - 1);
+    unsigned last = 0;
+    if (lane == 0) last = atomicAdd(p.tickets + bg, 1u) == (unsigned)(w_last - w_first);
+    last = __shfl_sync(kFull, last, 0);
+    if (!last) return;
+    __threadfence();
+    for (int idx = lane; idx < G * D; idx += 32) {
+      const int r = idx / D, d = idx - r * D;
+      float ms = -INFINITY;
+      for (int w = w_first; w <= w_last; ++w) ms = fmaxf(ms, __ldcg(p.partials + (long long)(w + bg) * rs + r * (D + 2)));
+      float ov = 0.f, lv = 0.f;
+      if (ms != -INFINITY) {
+        for (int w = w_first; w <= w_last; ++w) {
+          const float* st = p.partials + (long long)(w + bg) * rs + r * (D + 2);
+          const float f = ex2(__ldcg(st) - ms);
+          lv = fmaf(__ldcg(st + 1), f, lv);
+          ov = fmaf(__ldcg(st + 2 + d), f, ov);
+        }
+      }
+      p.out[((long long)b * p.Hq + g * G + r) * D + d] = lv > 0.f ? ov / lv : 0.f;
+    }
+    if (lane == 0) p.tickets[bg] = 0u;
+  }
+
+  // ---------------------------------------------------------- Q . K^T
+  __device__ __forceinline__ void qk_ternary(const unsigned char* kg, float (&s)[4]) {
+    uint32_t wa[S::kWPT], wb[S::kWPT];
+    const unsigned char* ra = kg + gid * (D / 4) + 4 * tig * S::kWPT;
+    const unsigned char* rb = kg + (gid + 8) * (D / 4) + 4 * tig * S::kWPT;
+    if constexpr (S::kWPT == 1) {
+      wa[0] = lds<uint32_t>(ra); wb[0] = lds<uint32_t>(rb);
+    } else if constexpr (S::kWPT == 2) {
+      const uint2 a = lds<uint2>(ra), b = lds<uint2>(rb);
+      wa[0] = a.x; wa[1] = a.y; wb[0] = b.x; wb[1] = b.y;
+    } else {
+      const uint4 a = lds<uint4>(ra), b = lds<uint4>(rb);
+      wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
+      wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
+    }
+    s[0] = s[1] = s[2] = s[3] = 0.f;
+#pragma unroll
+    for (int st = 0; st < S::kSteps; ++st) {
+      const int r0 = 2 * st, r1 = 2 * st + 1;
+      const int w0 = r0 >> 3, o0 = 2 * (r0 & 7), w1 = r1 >> 3, o1 = 2 * (r1 & 7);
+      mma16816(s, tern2(wa[w0], o0), tern2(wb[w0], o0), tern2(wa[w1], o1), tern2(wb[w1], o1),
+               qf[r0], qf[r1]);
+    }
+  }
+
+  __device__ __forceinline__ void qk_fp8(const unsigned char* kg, float (&s)[4]) {
+    s[0] = s[1] = s[2] = s[3] = 0.f;
+#pragma unroll
+    for (int wl = 0; wl < S::kWPT; ++wl) {
+      const uint4 xa = lds<uint4>(kg + gid * D + 16 * (tig * S::kWPT + wl));
+      const uint4 xb = lds<uint4>(kg + (gid + 8) * D + 16 * (tig * S::kWPT + wl));
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {         // k-step st = 4 * wl + q4, dims j = 2*q4, 2*q4+1
+        const int j = 2 * q4;
+        const uint32_t sel = sel_pair(j & 3);
+        const uint32_t pa = prmt(j < 4 ? xa.x : xa.y, j < 4 ? xa.z : xa.w, sel);
+        const uint32_t pb = prmt(j < 4 ? xb.x : xb.y, j < 4 ? xb.z : xb.w, sel);
+        const int st = 4 * wl + q4;
+        mma16816(s, e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16),
+                 qf[2 * st], qf[2 * st + 1]);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void qk_bf16(const unsigned char* kg, float (&s)[4]) {
+    s[0] = s[1] = s[2] = s[3] = 0.f;
+#pragma unroll
+    for (int wl = 0; wl < S::kWPT; ++wl) {
+      const unsigned char* ra = kg + gid * 2 * D + 32 * (tig * S::kWPT + wl);
+      const unsigned char* rb = kg + (gid + 8) * 2 * D + 32 * (tig * S::kWPT + wl);
+      const uint4 a0 = lds<uint4>(ra), a1 = lds<uint4>(ra + 16);
+      const uint4 b0 = lds<uint4>(rb), b1 = lds<uint4>(rb + 16);
+      const uint32_t ya[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t yb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {         // dims j = 2*q4 (+8) and 2*q4+1 (+8)
+        const int st = 4 * wl + q4;
+        mma16816(s, bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x5410u)), bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x5410u)),
+                 bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x7632u)), bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)),
+                 qf[2 * st], qf[2 * st + 1]);
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ P . V
+  // Token-pair masks for a partial page (tokens >= nt contribute nothing).
+  __device__ __forceinline__ void pv_masks(int nt, uint32_t& m01, uint32_t& m23) {
+    const int t0 = 2 * tig;
+    m01 = (t0 < nt ? 0x0000FFFFu : 0u) | (t0 + 1 < nt ? 0xFFFF0000u : 0u);
+    m23 = (t0 + 8 < nt ? 0x0000FFFFu : 0u) | (t0 + 9 < nt ? 0xFFFF0000u : 0u);
+  }
+
+  __device__ __forceinline__ void pv_ternary(const unsigned char* vg, uint32_t b0, uint32_t b1, int nt) {
+    const int t0 = 2 * tig;
+    const int vw0 = (gid * S::kUPT) >> 1;
+    uint32_t w0[S::kVW], w1[S::kVW], w2[S::kVW], w3[S::kVW];
+#pragma unroll
+    for (int i = 0; i < S::kVW; ++i) {
+      w0[i] = lds<uint32_t>(vg + t0 * (D / 4) + 4 * (vw0 + i));
+      w1[i] = lds<uint32_t>(vg + (t0 + 1) * (D / 4) + 4 * (vw0 + i));
+      w2[i] = lds<uint32_t>(vg + (t0 + 8) * (D / 4) + 4 * (vw0 + i));
+      w3[i] = lds<uint32_t>(vg + (t0 + 9) * (D / 4) + 4 * (vw0 + i));
+    }
+    uint32_t r01[S::kUPT], r23[S::kUPT];
+#pragma unroll
+    for (int ul = 0; ul < S::kUPT; ++ul) {
+      const int gu = gid * S::kUPT + ul;
+      const int wi = (gu >> 1) - vw0;
+      const uint32_t sel = (gu & 1) ? 0x7632u : 0x5410u;
+      r01[ul] = prmt(w0[wi], w1[wi], sel);
+      r23[ul] = prmt(w2[wi], w3[wi], sel);
+    }
+    if (nt < kPage) {
+      uint32_t m01, m23;
+      pv_masks(nt, m01, m23);
+#pragma unroll
+      for (int ul = 0; ul < S::kUPT; ++ul) { r01[ul] &= m01; r23[ul] &= m23; }
+    }
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt) {
+      const int la = mt, lb = mt + S::kSteps;
+      const int ua = la >> 3, ja = la & 7, ub = lb >> 3, jb = lb & 7;
+      mma16816(acc[mt], tern2(r01[ua], 2 * ja), tern2(r01[ub], 2 * jb), tern2(r23[ua], 2 * ja),
+               tern2(r23[ub], 2 * jb), b0, b1);
+    }
+  }
+
+  __device__ __forceinline__ void pv_fp8(const unsigned char* vg, uint32_t b0, uint32_t b1, int nt) {
+    const int t0 = 2 * tig;
+    constexpr int NWD = 2 * S::kUPT;          // u32 words of the thread's 8*kUPT bytes
+    uint32_t x0[NWD], x1[NWD], x2[NWD], x3[NWD];
+    const int off = 8 * gid * S::kUPT;
+#pragma unroll
+    for (int i = 0; i < NWD; i += 2) {
+      const uint2 a = lds<uint2>(vg + t0 * D + off + 4 * i);
+      const uint2 b = lds<uint2>(vg + (t0 + 1) * D + off + 4 * i);
+      const uint2 c = lds<uint2>(vg + (t0 + 8) * D + off + 4 * i);
+      const uint2 e = lds<uint2>(vg + (t0 + 9) * D + off + 4 * i);
+      x0[i] = a.x; x0[i + 1] = a.y; x1[i] = b.x; x1[i + 1] = b.y;
+      x2[i] = c.x; x2[i + 1] = c.y; x3[i] = e.x; x3[i + 1] = e.y;
+    }
+    uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
+    if (nt < kPage) pv_masks(nt, m01, m23);
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt) {
+      const int la = mt, lb = mt + S::kSteps;
+      const int ua = la >> 3, ja = la & 7, ub = lb >> 3, jb = lb & 7;
+      const int ia = 2 * ua + (ja >> 2), ib = 2 * ub + (jb >> 2);
+      const uint32_t sa = sel_pair(ja & 3) & 0xFFu, sb = sel_pair(jb & 3) & 0xFFu;
+      const uint32_t a0 = e4m3x2_f16(prmt(x0[ia], x1[ia], sa)) & m01;
+      const uint32_t a1 = e4m3x2_f16(prmt(x0[ib], x1[ib], sb)) & m01;
+      const uint32_t a2 = e4m3x2_f16(prmt(x2[ia], x3[ia], sa)) & m23;
+      const uint32_t a3 = e4m3x2_f16(prmt(x2[ib], x3[ib], sb)) & m23;
+      mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+
+  __device__ __forceinline__ void pv_bf16(const unsigned char* vg, uint32_t b0, uint32_t b1, int nt) {
+    const int t0 = 2 * tig;
+    const int off = 16 * gid * S::kUPT;       // bytes of the thread's dims in a row
+    uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
+    if (nt < kPage) pv_masks(nt, m01, m23);
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt) {
+      const int la = mt, lb = mt + S::kSteps;
+      const int ua = la >> 3, ja = la & 7, ub = lb >> 3, jb = lb & 7;
+      const int ba = off + 16 * ua + 4 * (ja >> 1), bb = off + 16 * ub + 4 * (jb >> 1);
+      const uint32_t sa = (ja & 1) ? 0x7632u : 0x5410u, sb = (jb & 1) ? 0x7632u : 0x5410u;
+      const uint32_t a0 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + ba), lds<uint32_t>(vg + (t0 + 1) * 2 * D + ba), sa)) & m01;
+      const uint32_t a1 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + bb), lds<uint32_t>(vg + (t0 + 1) * 2 * D + bb), sb)) & m01;
+      const uint32_t a2 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa)) & m23;
+      const uint32_t a3 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb)) & m23;
+      mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+
+  // --------------------------------------------------------- one entry
+  template <int FMT>
+  __device__ __forceinline__ void process(const unsigned char* e, const Desc& d) {
+    constexpr int CAP = FMT == KVC_FMT_TERNARY2 ? kMaxPages : (FMT == KVC_FMT_FP8_E4M3 ? 2 : 1);
+    constexpr int GB = group_bytes(FMT, D);
+    constexpr float KF = FMT == KVC_FMT_TERNARY2 ? 0.5f : 1.0f;   // ternary operands are 2c
+    const int np = d.np;
+    float s[CAP][4];
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) {
+      if (i < np) {
+        if constexpr (FMT == KVC_FMT_TERNARY2) qk_ternary(e + i * GB, s[i]);
+        else if constexpr (FMT == KVC_FMT_FP8_E4M3) qk_fp8(e + i * GB, s[i]);
+        else qk_bf16(e + i * GB, s[i]);
+      }
+    }
+    // scale, mask, entry maximum per column (cols 2*tig, 2*tig+1)
+    const bool c0ok = 2 * tig < p.G, c1ok = 2 * tig + 1 < p.G;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) {
+      if (i < np) {
+        const float sc = d.ks[i] * (KF * p.scale_log2);
+        const int nt = i == np - 1 ? d.ntok_last : kPage;
+        const bool r0 = gid < nt, r1 = gid + 8 < nt;
+        s[i][0] = (r0 && c0ok) ? s[i][0] * sc : -INFINITY;
+        s[i][1] = (r0 && c1ok) ? s[i][1] * sc : -INFINITY;
+        s[i][2] = (r1 && c0ok) ? s[i][2] * sc : -INFINITY;
+        s[i][3] = (r1 && c1ok) ? s[i][3] * sc : -INFINITY;
+        mx0 = fmaxf(mx0, fmaxf(s[i][0], s[i][2]));
+        mx1 = fmaxf(mx1, fmaxf(s[i][1], s[i][3]));
+      }
+    }
+    const bool need = mx0 > m0 + kTau || mx1 > m1 + kTau;
+    if (__any_sync(kFull, need)) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+      }
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float a0 = n0 == -INFINITY ? 1.f : ex2(m0 - n0);
+      const float a1 = n1 == -INFINITY ? 1.f : ex2(m1 - n1);
+#pragma unroll
+      for (int mt = 0; mt < S::kSteps; ++mt) {
+        acc[mt][0] *= a0; acc[mt][2] *= a0;
+        acc[mt][1] *= a1; acc[mt][3] *= a1;
+      }
+      l0 *= a0;
+      l1 *= a1;
+      m0 = n0;
+      m1 = n1;
+    }
+    // value-scale reference (warp-uniform: every lane reads the same desc)
+    constexpr float VF = FMT == KVC_FMT_TERNARY2 ? 0.5f : 1.0f;
+    float vmax = 0.f;
+#pragma unroll
+    for (int i = 0; i < CAP; ++i)
+      if (i < np) vmax = fmaxf(vmax, d.vs[i] * VF);
+    if (vmax > 0.f && (uref == 0.f || vmax > 16.f * uref || vmax < uref * 0.0625f)) {
+      const float beta = uref / vmax;
+#pragma unroll
+      for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[mt][c] *= beta;
+      uref = vmax;
+    }
+    const float inv_uref = uref > 0.f ? 1.f / uref : 0.f;
+    // P, row sums, P.V
+#pragma unroll
+    for (int i = 0; i < CAP; ++i) {
+      if (i < np) {
+        // padded GQA columns (>= G) have no finite maximum: keep them at 0
+        const float p00 = c0ok ? ex2(s[i][0] - m0) : 0.f, p01 = c1ok ? ex2(s[i][1] - m1) : 0.f;
+        const float p10 = c0ok ? ex2(s[i][2] - m0) : 0.f, p11 = c1ok ? ex2(s[i][3] - m1) : 0.f;
+        l0 += p00 + p10;
+        l1 += p01 + p11;
+        const float ratio = d.vs[i] * VF * inv_uref;
+        const uint32_t b0 = movtrans(f16x2(p00 * ratio, p01 * ratio));
+        const uint32_t b1 = movtrans(f16x2(p10 * ratio, p11 * ratio));
+        const int nt = i == np - 1 ? d.ntok_last : kPage;
+        const unsigned char* vg = e + S::kHalf + i * GB;
+        if constexpr (FMT == KVC_FMT_TERNARY2) pv_ternary(vg, b0, b1, nt);
+        else if constexpr (FMT == KVC_FMT_FP8_E4M3) pv_fp8(vg, b0, b1, nt);
+        else pv_bf16(vg, b0, b1, nt);
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- main
+  __device__ void run(int w_index, int n_warps, long long units) {
+    lane = threadIdx.x & 31;
+    gid = lane >> 2;
+    tig = lane & 3;
+    W = w_index;
+    nwg = n_warps;
+    U = units;
+    u0 = (long long)W * U / nwg;
+    u1 = (long long)(W + 1) * U / nwg;
+    cursor = u0;
+    cb = u0;
+    timed_out = false;
+    cur_bg = -1;
+    meta_phase_a(p, pr, cb + lane, u1, cur);
+    meta_phase_b(p, cur);
+    meta_phase_a(p, pr, cb + 32 + lane, u1, nxt);
+    nxt_b_pending = true;
+
+    bool issued[kEntries];
+#pragma unroll
+    for (int s = 0; s < kEntries; ++s) issued[s] = issue(s);
+    for (int it = 0;; ++it) {
+      const int slot = it % kEntries;
+      if (!issued[slot]) break;
+      if (!mbar_wait(&bars[slot], (uint32_t)((it / kEntries) & 1))) {
+        timed_out = true;
+        break;
+      }
+      const Desc& d = desc[slot];
+      const int fmt = d.fmt, bg = d.bg;
+      if (bg != cur_bg) {
+        finish();
+        begin(bg);
+      }
+      const unsigned char* e = ring + slot * S::kEntryBytes;
+      if (fmt == KVC_FMT_TERNARY2) process<KVC_FMT_TERNARY2>(e, d);
+      else if (fmt == KVC_FMT_FP8_E4M3) process<KVC_FMT_FP8_E4M3>(e, d);
+      else if (fmt == KVC_FMT_BF16) process<KVC_FMT_BF16>(e, d);
+      __syncwarp();
+      issued[slot] = issue(slot);
+    }
+    if (timed_out) {
+      if (lane == 0) atomicOr(p.err, kErrTimeout);
+      // let copies still in flight land before the CTA's memory is released
+      for (int s = 0; s < kEntries; ++s)
+        if (issued[s]) mbar_wait(&bars[s], 0u), mbar_wait(&bars[s], 1u);
+      return;
+    }
+    finish();
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) {
+  using S = Shape<D>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  unsigned char* ring = smem;
+  Desc* descs = reinterpret_cast<Desc*>(smem + kWarps * kEntries * S::kEntryBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(descs + kWarps * kEntries);
+  int* seqP = reinterpret_cast<int*>(bars + kWarps * kEntries);
+  int* seqL = seqP + (p.B + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x < kWarps * kEntries) mbar_init(&bars[threadIdx.x], 1);
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.B; base += 32) {
+      const int b = base + lane;
+      int u = 0;
+      if (b < p.B) {
+        int L = p.ctx[b];
+        if (L < 0 || L > p.max_pages * kPage) {
+          if (blockIdx.x == 0) atomicOr(p.err, kErrContext);
+          L = 0;
+        }
+        seqL[b] = L;
+        u = ((L + kPage - 1) / kPage) * p.Hkv;
+      }
+      int incl = u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+      }
+      if (b < p.B) seqP[b + 1] = carry + incl;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) seqP[0] = 0;
+  }
+  fence_mbar_init();
+  __syncthreads();
+  // sequences with nothing to attend to get a zero row
+  for (int b = blockIdx.x; b < p.B; b += gridDim.x)
+    if (seqL[b] == 0)
+      for (int i = threadIdx.x; i < p.Hq * D; i += blockDim.x) p.out[(long long)b * p.Hq * D + i] = 0.f;
+
+  const long long U = seqP[p.B];
+  if (U == 0) return;
+  const int nwg = (int)((long long)p.n_splits < U ? p.n_splits : U);   // n_splits = warps in the grid
+  const int W = blockIdx.x * kWarps + warp;
+  if (W >= nwg) return;
+  Worker<D> wk(p, Prologue{seqP, seqL}, ring + warp * kEntries * S::kEntryBytes, descs + warp * kEntries,
+               bars + warp * kEntries);
+  wk.run(W, nwg, U);
+}
+
+template <int D>
+size_t tc_smem_bytes(int batch) {
+  return (size_t)kWarps * kEntries * Shape<D>::kEntryBytes + kWarps * kEntries * sizeof(Desc) +
+         kWarps * kEntries * sizeof(uint64_t) + (size_t)(2 * batch + 1) * sizeof(int);
+}
+
+template <int D>
+cudaError_t tc_occupancy(int batch, int* ctas_per_sm) {
+  const size_t smem = tc_smem_bytes<D>(batch);
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D>, kWarps * 32, smem);
+}
+
+}  // namespace
+
+// Largest batch the tensor-core kernel handles (its per-CTA sequence table
+// lives in shared memory); larger batches use the CUDA-core kernel.
+constexpr int kTcMaxBatch = 1024;
+
+bool tc_supported(int batch, int hkv, int max_pages) {
+  return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages < (1ll << 31);
+}
+
+cudaError_t tc_grid(int batch, int d, int* grid) {
+  int dev = 0, sms = 0, per = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  switch (d) {
+    case 64: e = tc_occupancy<64>(batch, &per); break;
+    case 128: e = tc_occupancy<128>(batch, &per); break;
+    case 256: e = tc_occupancy<256>(batch, &per); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  *grid = sms * (per > 0 ? per : 1);
+  return cudaSuccess;
+}
+
+int tc_warps_per_cta() { return kWarps; }
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s) {
+  switch (head_dim) {
+    case 64: decode_tc_kernel<64><<<grid, kWarps * 32, tc_smem_bytes<64>(p.B), s>>>(p); break;
+    case 128: decode_tc_kernel<128><<<grid, kWarps * 32, tc_smem_bytes<128>(p.B), s>>>(p); break;
+    case 256: decode_tc_kernel<256><<<grid, kWarps * 32, tc_smem_bytes<256>(p.B), s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

@@ -36,13 +36,29 @@ kvc_status check_codec(const void* src, const void* dst, int n, int page_size, i
 namespace kvc {
 
 cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, DecodePlan* plan) {
+  const long long bg = (long long)batch * hkv;
+  const int G = hq / hkv;
+  const size_t record = (size_t)G * (d + 2) * sizeof(float);
+  plan->ticket_offset = 256;
+  plan->partial_offset = round_up(256 + (size_t)bg * 4, 256);
+  if (tc_supported(batch, hkv, max_pages)) {
+    // persistent grid, every warp a stream-K worker; one partial state per
+    // (warp, pair) boundary: at most warps + pairs records
+    int grid = 0;
+    cudaError_t e = tc_grid(batch, d, &grid);
+    if (e != cudaSuccess) return e;
+    plan->tensor_cores = true;
+    plan->grid = grid;
+    plan->n_splits = grid * tc_warps_per_cta();
+    plan->pages_per_split = 0;
+    plan->bytes = plan->partial_offset + ((size_t)plan->n_splits + (size_t)bg) * record;
+    return cudaSuccess;
+  }
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const long long bg = (long long)batch * hkv;
-  const int G = hq / hkv;
   // Split each (sequence, KV head) over pages so that about four CTAs per SM
   // are in flight, with at least 16 pages per split.
   long long splits = bg > 0 ? (4ll * sms + bg - 1) / bg : 1;
@@ -50,15 +66,16 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
   splits = std::max(1ll, std::min(splits, max_splits));
   const int pps = max_pages > 0 ? (int)((max_pages + splits - 1) / splits) : 1;
   splits = max_pages > 0 ? (max_pages + pps - 1) / pps : 1;
+  plan->tensor_cores = false;
+  plan->grid = 0;
   plan->n_splits = (int)splits;
   plan->pages_per_split = pps;
-  plan->ticket_offset = 256;
-  plan->partial_offset = round_up(256 + (size_t)bg * 4, 256);
-  plan->bytes = plan->partial_offset + (size_t)bg * splits * G * (d + 2) * sizeof(float);
+  plan->bytes = plan->partial_offset + (size_t)bg * splits * record;
   return cudaSuccess;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, const DecodePlan& plan, cudaStream_t s) {
+  if (plan.tensor_cores) return launch_decode_tc(p, head_dim, plan.grid, s);
   return launch_decode_simple(p, head_dim, s);
 }
 
@@ -237,7 +254,7 @@ kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache*
   p.err = reinterpret_cast<uint32_t*>(ws);
   p.tickets = reinterpret_cast<uint32_t*>(ws + plan.ticket_offset);
   p.partials = reinterpret_cast<float*>(ws + plan.partial_offset);
-  return from_cuda(kvc::launch_decode(p, head_dim, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(kvc::launch_decode(p, head_dim, plan, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kvc_status kvc_decode_read_error(void* workspace, int batch, int n_q_heads, int n_kv_heads,

@@ -60,15 +60,24 @@ struct DecodeParams {
 };
 
 struct DecodePlan {
-  int n_splits;
-  int pages_per_split;
+  bool tensor_cores;         // decode_tc kernel (else decode_simple)
+  int n_splits;              // simple: splits per (sequence, KV head); tc: warps in the grid
+  int pages_per_split;       // simple only
+  int grid;                  // tc only: persistent CTAs
   size_t ticket_offset, partial_offset, bytes;
 };
 
-// Split-K plan and workspace layout for these shapes on the current device.
+// Kernel choice, split-K plan and workspace layout for these shapes on the
+// current device.
 cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, DecodePlan* plan);
 
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, const DecodePlan& plan, cudaStream_t s);
 cudaError_t launch_decode_simple(const DecodeParams& p, int head_dim, cudaStream_t s);
+
+// tensor-core kernel (decode_tc.cu)
+bool tc_supported(int batch, int hkv, int max_pages);
+cudaError_t tc_grid(int batch, int d, int* grid);
+int tc_warps_per_cta();
+cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s);
 
 }  // namespace kvc

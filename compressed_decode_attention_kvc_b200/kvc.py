@@ -68,7 +68,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m compressed_decode_attention_kvc_b200.build`")
+            "`python compressed_decode_attention_kvc_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, f32, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int
     lib.kvc_status_string.restype = ctypes.c_char_p

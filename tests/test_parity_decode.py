@@ -81,6 +81,17 @@ def test_edge_lengths_and_windows(cuda_device):
         assert_attention_close(out, ref, f"sink={sink} window={window}")
 
 
+def test_large_batch_uses_cuda_core_kernel(cuda_device):
+    # more sequences than the tensor-core kernel's per-CTA sequence table
+    # holds: the CUDA-core kernel serves the call
+    inp = synth.make_decode_inputs("tiny", seed=6, batch=1100, context=16 * 3, window=8, n_q_heads=4,
+                                   n_kv_heads=2)
+    g = torch.Generator().manual_seed(3)
+    inp["context_lens"] = torch.randint(0, 16 * 3 + 1, (1100,), generator=g, dtype=torch.int32)
+    out, ref, _ = _decode_vs_oracle(inp, cuda_device)
+    assert_attention_close(out, ref, "batch 1100")
+
+
 def test_repeated_calls_reuse_workspace(cuda_device):
     inp = synth.make_decode_inputs("qwen3b", seed=4, batch=2, context=700)
     cfg = inp["cfg"]
