@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager launches instead of replaying a captured CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -219,6 +221,25 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # per-kernel device times: eager steps with an event pair around each launch
+    marks = []
+    for _ in range(min(args.steps, 20)):
+        step(marks)
+    torch.cuda.synchronize()
+    per_kernel = {}
+    for name, e0, e1 in marks:
+        per_kernel.setdefault(name, []).append(e0.elapsed_time(e1))
+    # the timed steps replay one captured step (a CUDA graph), so host-side
+    # launch overhead is not in the measurement
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -226,12 +247,14 @@ def run_ours(args, rank, world, dev, peak, peak_src):
                           else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])
     clocks.start()
     time.sleep(0.3)
-    marks = []
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        step(marks)
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -239,9 +262,7 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     torch.cuda.synchronize()
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
-    per_kernel = {}
-    for name, e0, e1 in marks:
-        per_kernel.setdefault(name, []).append(e0.elapsed_time(e1))
+    del graph
     flags = K.kvc_decode_read_error(ws, B, hq, H, D, max_pages)
     if flags:
         raise RuntimeError(f"device error flags {flags}")
@@ -430,6 +451,9 @@ def config_block(args, cfg):
             "page_size": P, "step": "pack every page of the batch into its format (bf16 copy / fp8 / "
                                     "ternary) + one decode-attention pass over the compressed cache",
             "l2": "inputs larger than L2 (bf16 source pages of the batch exceed 126 MB)",
+            "timing": ("CUDA events around K eager steps" if args.eager else
+                       "CUDA events around K replays of one captured step (CUDA graph)")
+                      + "; per-kernel times from event pairs around each launch in eager steps",
             "parallelism": f"dp{args.gpus} (independent batch per GPU)"}
 
 

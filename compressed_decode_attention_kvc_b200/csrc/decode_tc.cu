@@ -9,13 +9,16 @@
 //
 // Design (B200):
 // * Work: the (sequence, KV head, page) units of the whole batch are split
-//   evenly over every warp of a persistent grid ("stream-K"): warp W owns
-//   units [W*U/NW, (W+1)*U/NW), which may span several (sequence, KV head)
-//   pairs.  Each warp is an independent worker; no CTA-wide synchronisation
-//   after the prologue.  Ragged context lengths balance by construction.
-// * Staging: each warp keeps a 2-entry ring in shared memory; an entry holds
-//   up to 8 ternary pages, 2 FP8 pages or 1 BF16 page (K group then V group
-//   of one KV head), filled with 1-D TMA bulk copies (cp.async.bulk, no
+//   over every warp of a persistent grid ("stream-K"), weighted by the bytes
+//   each page moves (a BF16 page of the window costs 8 ternary pages): warp
+//   W owns the units whose weighted start lies in [W*C/NW, (W+1)*C/NW), a
+//   range that may span several (sequence, KV head) pairs.  Each warp is an
+//   independent worker; no CTA-wide synchronisation after the prologue.
+//   Ragged context lengths and format mixes balance by construction.
+// * Staging: each warp keeps a 2-entry ring in shared memory; an 8 KB entry
+//   (4 KB at head_dim 64) holds the K groups then the V groups of up to 8
+//   ternary pages, 2 FP8 pages or one BF16 page (half a page at head_dim
+//   256) of one KV head, filled with 1-D TMA bulk copies (cp.async.bulk, no
 //   multicast) that complete on an mbarrier.  Page metadata (format, block-
 //   table slot, scales) for 32 units at a time is loaded lane-parallel one
 //   chunk ahead, so the warp never waits on a dependent global load.
@@ -28,10 +31,10 @@
 //   exactly, 00 is 0.  FP8 pages convert with cvt.f16x2.e4m3x2, BF16 pages
 //   with a byte permute and cvt.f16x2.f32.  Tensor-core operands come from
 //   registers, so no unpacked copy of a page ever touches shared memory.
-// * Softmax: online, in log2 units, with a lazy maximum: the running maximum
-//   moves (and the accumulators are rescaled) only when a score exceeds it
-//   by more than 2^8, so P stays within f16 range without a cross-lane max
-//   on every page.  Per-page V scales are folded into P relative to a
+// * Softmax: online, per page, in log2 units, with a lazy maximum: the
+//   running maximum moves (and the accumulators are rescaled) only when a
+//   score exceeds it by more than 2^8, so P stays within f16 range without a
+//   cross-lane max on every page.  Per-page V scales are folded into P relative to a
 //   per-warp reference scale that is re-based when the ratio leaves
 //   [1/16, 16], keeping P far from the f16 subnormal range.
 // * Merge: each warp writes one partial state per (sequence, KV head) it
@@ -41,30 +44,42 @@
 
 #include <math.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 namespace kvc {
 namespace {
 
+constexpr int kTcMaxBatchTpl = 1024;   // largest batch of the tensor-core kernel
+
 constexpr int kWarps = 4;            // warps per CTA; each is an independent worker
 constexpr int kEntries = 2;          // ring entries per warp
-constexpr int kMaxPages = 8;         // pages per entry (ternary)
+constexpr int kMaxPages = 8;         // pages per entry
 constexpr float kTau = 8.0f;         // lazy-max threshold, log2 units
 constexpr uint32_t kSpinLimit = 1u << 22;
 constexpr int kSkip = 3;             // entry carrying an unusable page (flagged, no data)
 constexpr unsigned kFull = 0xffffffffu;
+// Work weights of one page of one KV head, proportional to the bytes it moves.
+constexpr int kCostTern = 1, kCostFp8 = 4, kCostBf16 = 8;
 
 struct Desc {
-  int fmt, np, bg, ntok_last;
+  int fmt, np, bg, nrows;            // nrows: valid token rows of the entry's last page
+  int row0;                          // first page row held (BF16 half pages: 0 or 8)
   float ks[kMaxPages], vs[kMaxPages];
 };
 
 template <int D>
 struct Shape {
-  static constexpr int kEntryBytes = 64 * D;   // one BF16 page: K group + V group
-  static constexpr int kHalf = 32 * D;         // K region | V region of an entry
-  static constexpr int kSteps = D / 16;        // k-steps of Q.K^T = m-tiles of P.V
-  static constexpr int kWPT = D / 64;          // K words (16 dims) per thread per token
-  static constexpr int kUPT = D / 64;          // V units (8 dims) per thread
-  static constexpr int kVW = kUPT > 1 ? kUPT / 2 : 1;   // V code words per thread per token
+  static constexpr int kEntryBytes = D == 64 ? 4096 : 8192;
+  static constexpr int kHalf = kEntryBytes / 2;            // K region | V region
+  static constexpr int kSteps = D / 16;                    // k-steps of Q.K^T = m-tiles of P.V
+  static constexpr int kWPT = D / 64;                      // K words (16 dims) per thread per token
+  static constexpr int kUPT = D / 64;                      // V units (8 dims) per thread
+  static constexpr int kVW = kUPT > 1 ? kUPT / 2 : 1;      // V code words per thread per token
+  static constexpr int kTernCap = kHalf / (4 * D) < kMaxPages ? kHalf / (4 * D) : kMaxPages;
+  static constexpr int kFp8Cap = kHalf / (16 * D);
+  static constexpr int kBf16Rows = kHalf / (2 * D) >= 16 ? 16 : 8;   // token rows of a BF16 page per entry
 };
 
 __host__ __device__ constexpr int group_bytes(int fmt, int d) {
@@ -157,79 +172,143 @@ __device__ __forceinline__ T lds(const unsigned char* p) {
   return *reinterpret_cast<const T*>(p);
 }
 
-// ------------------------------------------------------------- metadata
-struct Meta {          // one unit (page of one KV head), held by one lane
-  int fmt;             // page format, or kSkip when unusable
-  int phys;            // slot in the pool of that format
-  int bg;              // b * Hkv + g
-  int ntok;            // valid tokens of the page (1..16)
-  float ks, vs;        // K / V scale of the page (gamma, s, or 1)
-  int older;           // caller tag (phase A) before fmt is resolved
-  int j, L;            // page index, sequence length
+// ------------------------------------------------------- work partition
+// Sequence b contributes Hkv * np(b) units (page of one KV head), ordered
+// (b, g, j).  Each unit carries a weight: the high-precision format's cost
+// for sink and window pages, the ternary cost for older pages (anchors are
+// counted as ternary).  Warp W of NW owns the units whose weighted start
+// lies in [W*C/NW, (W+1)*C/NW), C the total weight.
+struct SeqShape {
+  int np, ns, jw2, cost;   // pages, sink pages, first window page (>= ns), weight per KV head
 };
+
+__device__ __forceinline__ SeqShape seq_shape(int L, int sink, int window, int whp) {
+  SeqShape s;
+  s.np = (L + kPage - 1) / kPage;
+  s.ns = min(s.np, (sink + kPage - 1) / kPage);
+  int jw = s.np;
+  if (window > 0) jw = L - window > 0 ? (L - window) / kPage : 0;
+  s.jw2 = max(s.ns, min(jw, s.np));
+  s.cost = whp * (s.ns + (s.np - s.jw2)) + (s.jw2 - s.ns) * kCostTern;
+  return s;
+}
+// weighted start of page j inside one (sequence, KV head)
+__device__ __forceinline__ int cost_of_page(const SeqShape& s, int j, int whp) {
+  if (j <= s.ns) return whp * j;
+  if (j <= s.jw2) return whp * s.ns + (j - s.ns);
+  return whp * s.ns + (s.jw2 - s.ns) + whp * (j - s.jw2);
+}
+// first page whose weighted start is >= c (np when none)
+__device__ __forceinline__ int page_of_cost(const SeqShape& s, int c, int whp) {
+  const int a = whp * s.ns;
+  if (c <= a) return (c + whp - 1) / whp;
+  const int bnd = a + (s.jw2 - s.ns);
+  if (c <= bnd) return s.ns + (c - a);
+  return min(s.np, s.jw2 + (c - bnd + whp - 1) / whp);
+}
 
 struct Prologue {
-  const int* seqP;     // [B + 1] unit prefix over sequences
+  const int* seqP;     // [B + 1] unit prefix
+  const int* seqC;     // [B + 1] weight prefix
   const int* seqL;     // [B] validated lengths
+  int B, Hkv, sink, window, whp;
+  long long C;         // total weight
+  int U;               // total units
+  int nwg;             // workers in the partition
+
+  // last b with prefix[b] <= x (prefix nondecreasing, x < prefix[B])
+  __device__ __forceinline__ int find(const int* prefix, long long x) const {
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= x) lo = mid; else hi = mid;
+    }
+    return lo;
+  }
+  // first unit whose weighted start is >= c
+  __device__ int unit_of_cost(long long c) const {
+    if (c >= C) return U;
+    const int b = find(seqC, c);
+    const SeqShape s = seq_shape(seqL[b], sink, window, whp);
+    const int cl = (int)(c - seqC[b]);
+    const int g = cl / s.cost;
+    const int j = page_of_cost(s, cl - g * s.cost, whp);
+    return seqP[b] + g * s.np + j;
+  }
+  // worker that owns unit x
+  __device__ int worker_of(int x) const {
+    const int b = find(seqP, x);
+    const SeqShape s = seq_shape(seqL[b], sink, window, whp);
+    const int off = x - seqP[b];
+    const int g = off / s.np;
+    const long long cs = seqC[b] + (long long)g * s.cost + cost_of_page(s, off - g * s.np, whp);
+    return (int)(((cs + 1) * nwg + C - 1) / C) - 1;
+  }
 };
 
-// Phase A: unit -> (sequence, KV head, page); block-table slot and caller tag.
-__device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prologue& pr, long long x,
-                                             long long u1, Meta& m) {
-  m.fmt = kSkip;
-  m.phys = -1;
-  m.bg = -1;
-  m.ntok = 0;
-  m.ks = m.vs = 0.f;
-  m.older = KVC_FMT_TERNARY2;
-  m.j = 0;
-  m.L = 0;
+// ------------------------------------------------------------- metadata
+// Per-lane page metadata, packed: fmt (2 bits) | nrows (5 bits) << 2 | bg << 7.
+__device__ __forceinline__ int meta_pack(int fmt, int ntok, int bg) { return fmt | (ntok << 2) | (bg << 7); }
+__device__ __forceinline__ int meta_fmt(int m) { return m & 3; }
+__device__ __forceinline__ int meta_ntok(int m) { return (m >> 2) & 31; }
+__device__ __forceinline__ int meta_bg(int m) { return m >> 7; }
+
+struct MetaA {    // after the block-table load
+  int phys, older, bg, j;   // bg < 0: no unit
+};
+struct Meta {     // resolved
+  int m;          // packed fmt / ntok / bg (bg = -1 encoded as m < 0)
+  int phys;
+  float ks, vs;
+};
+
+__device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prologue& pr, int x, int u1,
+                                             MetaA& a) {
+  a.bg = -1;
+  a.phys = 0;
+  a.older = KVC_FMT_TERNARY2;
+  a.j = 0;
   if (x >= u1) return;
-  int lo = 0, hi = p.B;          // seqP[lo] <= x < seqP[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pr.seqP[mid] <= x) lo = mid; else hi = mid;
-  }
-  const int b = lo;
-  const int L = pr.seqL[b];
-  const int np = (L + kPage - 1) / kPage;
-  const int off = (int)(x - pr.seqP[b]);
+  const int b = pr.find(pr.seqP, x);
+  const int np = (pr.seqL[b] + kPage - 1) / kPage;
+  const int off = x - pr.seqP[b];
   const int g = off / np;
   const int j = off - g * np;
   const long long row = (long long)b * p.max_pages + j;
-  m.bg = b * p.Hkv + g;
-  m.j = j;
-  m.L = L;
-  m.ntok = min(kPage, L - j * kPage);
-  m.phys = __ldg(p.block_table + row);
-  m.older = p.older_fmt ? (int)__ldg(p.older_fmt + row) : KVC_FMT_TERNARY2;
+  a.bg = b * p.Hkv + g;
+  a.j = j;
+  a.phys = __ldg(p.block_table + row);
+  a.older = p.older_fmt ? (int)__ldg(p.older_fmt + row) : KVC_FMT_TERNARY2;
 }
 
-// Phase B: resolve the format, check the slot, load the scales.
-__device__ __forceinline__ void meta_phase_b(const DecodeParams& p, Meta& m) {
-  if (m.bg < 0) return;
-  const int fmt = page_format(m.j, m.L, p.sink, p.window, p.hp, m.older);
+__device__ __forceinline__ void meta_phase_b(const DecodeParams& p, const Prologue& pr, const MetaA& a,
+                                             Meta& m) {
+  m.ks = m.vs = 0.f;
+  m.phys = a.phys;
+  if (a.bg < 0) {
+    m.m = -1;
+    return;
+  }
+  const int b = a.bg / p.Hkv, g = a.bg - b * p.Hkv;
+  const int L = pr.seqL[b];
+  const int ntok = min(kPage, L - a.j * kPage);
+  int fmt = page_format(a.j, L, p.sink, p.window, p.hp, a.older);
   if (fmt < 0 || fmt > 2) {
     atomicOr(p.err, kErrFormat);
-    m.fmt = kSkip;
-    return;
-  }
-  if (m.phys < 0 || m.phys >= p.cache.n_pages[fmt]) {
+    fmt = kSkip;
+  } else if (a.phys < 0 || a.phys >= p.cache.n_pages[fmt]) {
     atomicOr(p.err, kErrBlockTable);
-    m.fmt = kSkip;
-    return;
-  }
-  m.fmt = fmt;
-  const int g = m.bg % p.Hkv;
-  if (fmt == KVC_FMT_TERNARY2) {
-    m.ks = __ldg(p.cache.k_gamma + (long long)m.phys * p.Hkv + g);
-    m.vs = __ldg(p.cache.v_gamma + (long long)m.phys * p.Hkv + g);
+    fmt = kSkip;
+  } else if (fmt == KVC_FMT_TERNARY2) {
+    m.ks = __ldg(p.cache.k_gamma + (long long)a.phys * p.Hkv + g);
+    m.vs = __ldg(p.cache.v_gamma + (long long)a.phys * p.Hkv + g);
   } else if (fmt == KVC_FMT_FP8_E4M3) {
-    m.ks = __ldg(p.cache.k_fp8_scale + m.phys);
-    m.vs = __ldg(p.cache.v_fp8_scale + m.phys);
+    m.ks = __ldg(p.cache.k_fp8_scale + a.phys);
+    m.vs = __ldg(p.cache.v_fp8_scale + a.phys);
   } else {
     m.ks = m.vs = 1.f;
   }
+  m.m = meta_pack(fmt, ntok, a.bg);
 }
 
 // ----------------------------------------------------------- the worker
@@ -237,62 +316,85 @@ template <int D>
 struct Worker {
   using S = Shape<D>;
   const DecodeParams& p;
-  const Prologue pr;
+  const Prologue& pr;
   unsigned char* ring;     // this warp's kEntries entries
   Desc* desc;              // [kEntries]
   uint64_t* bars;          // [kEntries]
   int lane, gid, tig;
-  long long u0, u1, cursor, cb;   // unit range, next unit to issue, chunk base
+  int u1, cursor, cb;      // unit range end, next unit to issue, chunk base
+  int bf16_half;           // next half of a BF16 page to issue (half-page entries)
   Meta cur, nxt;
+  MetaA nxa;
   bool nxt_b_pending;
-  int W, nwg;
-  long long U;
-  bool timed_out;
+  int W;
 
   // per (sequence, KV head) state
   int cur_bg;
   uint32_t qf[2 * S::kSteps];
   float acc[S::kSteps][4];
-  float m0, m1, l0, l1, uref;
+  float m0, m1, l0, l1, uref, inv_uref;
 
-  __device__ Worker(const DecodeParams& pp, Prologue prr, unsigned char* r, Desc* d, uint64_t* b)
+  __device__ Worker(const DecodeParams& pp, const Prologue& prr, unsigned char* r, Desc* d, uint64_t* b)
       : p(pp), pr(prr), ring(r), desc(d), bars(b) {}
 
   __device__ __forceinline__ int shfl(int v, int src) { return __shfl_sync(kFull, v, src); }
+  __device__ __forceinline__ float shflf(float v, int src) { return __shfl_sync(kFull, v, src); }
 
-  // Fill ring slot `slot` with the next entry.  Returns false when the
-  // warp's units are exhausted.
+  // Fill ring slot `slot` with the next entry; false when the warp's units
+  // are exhausted.
   __device__ bool issue(int slot) {
     if (cursor >= u1) return false;
-    int li = (int)(cursor - cb);
+    int li = cursor - cb;
     if (li >= 32) {
-      if (nxt_b_pending) meta_phase_b(p, nxt);
+      if (nxt_b_pending) meta_phase_b(p, pr, nxa, nxt);
       cur = nxt;
       cb += 32;
       li -= 32;
-      meta_phase_a(p, pr, cb + 32 + lane, u1, nxt);
+      meta_phase_a(p, pr, cb + 32 + lane, u1, nxa);
       nxt_b_pending = true;
     } else if (nxt_b_pending) {
-      meta_phase_b(p, nxt);
+      meta_phase_b(p, pr, nxa, nxt);
       nxt_b_pending = false;
     }
-    const int f0 = shfl(cur.fmt, li);
-    const int bg0 = shfl(cur.bg, li);
-    int np = 1;
-    if (f0 != kSkip) {
-      const int cap = f0 == KVC_FMT_TERNARY2 ? kMaxPages : (f0 == KVC_FMT_FP8_E4M3 ? 2 : 1);
-      const bool ok = lane >= li && (cb + lane) < u1 && cur.fmt == f0 && cur.bg == bg0;
-      const uint32_t run = __ballot_sync(kFull, ok) >> li;
-      const int len = (run == 0xffffffffu) ? 32 : __ffs(~run) - 1;
-      np = min(len, cap);
+    const int m0l = shfl(cur.m, li);
+    const int f0 = meta_fmt(m0l), bg0 = meta_bg(m0l);
+    int np = 1, row0 = 0, nrows, advance = 1;
+    int bytes_per_page = 0, src_off = 0;
+    if (f0 == KVC_FMT_BF16 && S::kBf16Rows == 8) {
+      // a BF16 page of this head size fills two entries of 8 token rows
+      const int ntok = meta_ntok(m0l);
+      row0 = 8 * bf16_half;
+      nrows = min(8, ntok - row0);
+      bytes_per_page = 8 * 2 * D;
+      src_off = row0 * 2 * D;
+      if (bf16_half == 0 && ntok > 8) {
+        bf16_half = 1;
+        advance = 0;
+      } else {
+        bf16_half = 0;
+      }
+    } else {
+      if (f0 != kSkip) {
+        const int cap = f0 == KVC_FMT_TERNARY2 ? S::kTernCap : (f0 == KVC_FMT_FP8_E4M3 ? S::kFp8Cap : 1);
+        // only the last page of a (sequence, KV head) can be partial, and it
+        // ends the run, so every page but the entry's last is full
+        const bool ok = lane >= li && (cb + lane) < u1 && cur.m >= 0 && meta_fmt(cur.m) == f0 &&
+                        meta_bg(cur.m) == bg0;
+        const uint32_t run = __ballot_sync(kFull, ok) >> li;
+        const int len = (run == 0xffffffffu) ? 32 : __ffs(~run) - 1;
+        np = max(1, min(len, cap));
+        bytes_per_page = group_bytes(f0, D);
+      }
+      advance = np;
+      nrows = meta_ntok(shfl(cur.m, min(li + np - 1, 31)));
     }
-    const int ntok_last = shfl(cur.ntok, min(li + np - 1, 31));
     Desc& d = desc[slot];
     if (lane == li) {
       d.fmt = f0;
       d.np = np;
       d.bg = bg0;
-      d.ntok_last = ntok_last;
+      d.nrows = nrows;
+      d.row0 = row0;
     }
     if (lane >= li && lane < li + np) {
       d.ks[lane - li] = cur.ks;
@@ -303,12 +405,12 @@ struct Worker {
     if (f0 == kSkip) {
       if (lane == 0) mbar_arrive_expect_tx(&bars[slot], 0);
     } else {
-      const int gb = group_bytes(f0, D);
-      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(2 * np * gb));
+      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(2 * np * bytes_per_page));
       __syncwarp();
       if (lane >= li && lane < li + np) {
         const int k = lane - li;
-        const int g = cur.bg % p.Hkv;
+        const int g = bg0 % p.Hkv;
+        const int gb = group_bytes(f0, D);
         const long long grp = (long long)cur.phys * p.Hkv + g;
         const unsigned char* ksrc;
         const unsigned char* vsrc;
@@ -323,17 +425,14 @@ struct Worker {
           vsrc = static_cast<const unsigned char*>(p.cache.v_bf16);
         }
         unsigned char* e = ring + slot * S::kEntryBytes;
-        bulk_g2s(e + k * gb, ksrc + grp * gb, (uint32_t)gb, &bars[slot]);
-        bulk_g2s(e + S::kHalf + k * gb, vsrc + grp * gb, (uint32_t)gb, &bars[slot]);
+        bulk_g2s(e + k * bytes_per_page, ksrc + grp * gb + src_off, (uint32_t)bytes_per_page, &bars[slot]);
+        bulk_g2s(e + S::kHalf + k * bytes_per_page, vsrc + grp * gb + src_off, (uint32_t)bytes_per_page,
+                 &bars[slot]);
       }
     }
     __syncwarp();
-    cursor += np;
+    cursor += advance;
     return true;
-  }
-
-  __device__ __forceinline__ int warp_of(long long x) const {
-    return (int)(((x + 1) * (long long)nwg + U - 1) / U) - 1;
   }
 
   // Start a new (sequence, KV head): load Q as f16 B fragments, reset state.
@@ -354,7 +453,7 @@ struct Worker {
 #pragma unroll
       for (int i = 0; i < S::kWPT * 8; ++i) raw[i] = 0u;
     }
-    // qf[ri] = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) + (ri & 7) (local dims)
+    // qf[ri] = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) + (ri & 7) (thread-local dims)
 #pragma unroll
     for (int ri = 0; ri < 2 * S::kSteps; ++ri) {
       const int wl = ri >> 3, j = ri & 7;
@@ -368,6 +467,7 @@ struct Worker {
     m0 = m1 = -INFINITY;
     l0 = l1 = 0.f;
     uref = 0.f;
+    inv_uref = 0.f;
   }
 
   // Write this warp's partial state for cur_bg; the last writer merges.
@@ -405,32 +505,89 @@ struct Worker {
     __syncwarp();
     const int b = bg / p.Hkv, g = bg - b * p.Hkv;
     const int np = (pr.seqL[b] + kPage - 1) / kPage;
-    const long long sbg = pr.seqP[b] + (long long)g * np;
-    const int w_first = warp_of(sbg), w_last = warp_of(sbg + np - 1);
+    const int x0 = pr.seqP[b] + g * np;
+    const int w_first = pr.worker_of(x0), w_last = pr.worker_of(x0 + np - 1);
     unsigned last = 0;
     if (lane == 0) last = atomicAdd(p.tickets + bg, 1u) == (unsigned)(w_last - w_first);
     last = __shfl_sync(kFull, last, 0);
     if (!last) return;
     __threadfence();
-    for (int idx = lane; idx < G * D; idx += 32) {
-      const int r = idx / D, d = idx - r * D;
-      float ms = -INFINITY;
-      for (int w = w_first; w <= w_last; ++w) ms = fmaxf(ms, __ldcg(p.partials + (long long)(w + bg) * rs + r * (D + 2)));
-      float ov = 0.f, lv = 0.f;
-      if (ms != -INFINITY) {
-        for (int w = w_first; w <= w_last; ++w) {
-          const float* st = p.partials + (long long)(w + bg) * rs + r * (D + 2);
-          const float f = ex2(__ldcg(st) - ms);
-          lv = fmaf(__ldcg(st + 1), f, lv);
-          ov = fmaf(__ldcg(st + 2 + d), f, ov);
+    merge(bg, w_first, w_last);
+  }
+
+  // Merge the partial states of one (sequence, KV head) and write its output
+  // rows.  Records are read with independent loads: per-record weights
+  // lane-parallel (lane k owns record k of a batch of 32), then float4 rows.
+  __device__ void merge(int bg, int w_first, int w_last) {
+    const int G = p.G;
+    const int rs = G * (D + 2);
+    const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+    const int nrec = w_last - w_first + 1;
+    // row maxima and normalisers
+    float ms[8], ls[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) { ms[r] = -INFINITY; ls[r] = 0.f; }
+    for (int k0 = 0; k0 < nrec; k0 += 32) {
+      const int k = k0 + lane;
+      const float* st = p.partials + (long long)(w_first + k + bg) * rs;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        float mk = -INFINITY;
+        if (r < G && k < nrec) mk = __ldcg(st + r * (D + 2));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, o));
+        ms[r] = fmaxf(ms[r], mk);
+      }
+    }
+    for (int k0 = 0; k0 < nrec; k0 += 32) {
+      const int k = k0 + lane;
+      const float* st = p.partials + (long long)(w_first + k + bg) * rs;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        float lk = 0.f;
+        if (r < G && k < nrec && ms[r] != -INFINITY) lk = __ldcg(st + r * (D + 2) + 1) * ex2(__ldcg(st + r * (D + 2)) - ms[r]);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
+        ls[r] += lk;
+      }
+    }
+    // output rows: lane owns D/32 consecutive dims of every row
+    constexpr int DPL = D / 32;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r >= G) break;
+      float o[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) o[i] = 0.f;
+      if (ms[r] != -INFINITY) {
+        for (int k0 = 0; k0 < nrec; k0 += 32) {
+          const int k = k0 + lane;
+          float f = 0.f;
+          if (k < nrec) f = ex2(__ldcg(p.partials + (long long)(w_first + k + bg) * rs + r * (D + 2)) - ms[r]);
+          const int kn = min(32, nrec - k0);
+#pragma unroll 4
+          for (int kk = 0; kk < kn; ++kk) {
+            const float fk = __shfl_sync(kFull, f, kk);
+            const float* row = p.partials + (long long)(w_first + k0 + kk + bg) * rs + r * (D + 2) + 2 + lane * DPL;
+#pragma unroll
+            for (int i = 0; i < DPL; i += 2) {
+              const float2 v = __ldcg(reinterpret_cast<const float2*>(row + i));
+              o[i] = fmaf(fk, v.x, o[i]);
+              o[i + 1] = fmaf(fk, v.y, o[i + 1]);
+            }
+          }
         }
       }
-      p.out[((long long)b * p.Hq + g * G + r) * D + d] = lv > 0.f ? ov / lv : 0.f;
+      const float inv = ls[r] > 0.f ? 1.f / ls[r] : 0.f;
+      float* dst = p.out + ((long long)b * p.Hq + g * G + r) * D + lane * DPL;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) dst[i] = o[i] * inv;
     }
     if (lane == 0) p.tickets[bg] = 0u;
   }
 
   // ---------------------------------------------------------- Q . K^T
+  // two independent accumulation chains, summed at the end
   __device__ __forceinline__ void qk_ternary(const unsigned char* kg, float (&s)[4]) {
     uint32_t wa[S::kWPT], wb[S::kWPT];
     const unsigned char* ra = kg + gid * (D / 4) + 4 * tig * S::kWPT;
@@ -445,57 +602,69 @@ struct Worker {
       wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
       wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
     }
-    s[0] = s[1] = s[2] = s[3] = 0.f;
+    float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int st = 0; st < S::kSteps; ++st) {
       const int r0 = 2 * st, r1 = 2 * st + 1;
       const int w0 = r0 >> 3, o0 = 2 * (r0 & 7), w1 = r1 >> 3, o1 = 2 * (r1 & 7);
-      mma16816(s, tern2(wa[w0], o0), tern2(wb[w0], o0), tern2(wa[w1], o1), tern2(wb[w1], o1),
+      mma16816(t[st & 1], tern2(wa[w0], o0), tern2(wb[w0], o0), tern2(wa[w1], o1), tern2(wb[w1], o1),
                qf[r0], qf[r1]);
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) s[c] = t[0][c] + t[1][c];
   }
 
   __device__ __forceinline__ void qk_fp8(const unsigned char* kg, float (&s)[4]) {
-    s[0] = s[1] = s[2] = s[3] = 0.f;
+    float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int wl = 0; wl < S::kWPT; ++wl) {
       const uint4 xa = lds<uint4>(kg + gid * D + 16 * (tig * S::kWPT + wl));
       const uint4 xb = lds<uint4>(kg + (gid + 8) * D + 16 * (tig * S::kWPT + wl));
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {         // k-step st = 4 * wl + q4, dims j = 2*q4, 2*q4+1
+      for (int q4 = 0; q4 < 4; ++q4) {         // k-step 4*wl + q4: dims j, j+1 (and +8), j = 2*q4
         const int j = 2 * q4;
         const uint32_t sel = sel_pair(j & 3);
         const uint32_t pa = prmt(j < 4 ? xa.x : xa.y, j < 4 ? xa.z : xa.w, sel);
         const uint32_t pb = prmt(j < 4 ? xb.x : xb.y, j < 4 ? xb.z : xb.w, sel);
         const int st = 4 * wl + q4;
-        mma16816(s, e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16),
+        mma16816(t[st & 1], e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16),
                  qf[2 * st], qf[2 * st + 1]);
       }
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) s[c] = t[0][c] + t[1][c];
   }
 
+  // ROWS = token rows of the page held by the entry (16, or 8 for half pages)
+  template <int ROWS>
   __device__ __forceinline__ void qk_bf16(const unsigned char* kg, float (&s)[4]) {
-    s[0] = s[1] = s[2] = s[3] = 0.f;
+    float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int wl = 0; wl < S::kWPT; ++wl) {
       const unsigned char* ra = kg + gid * 2 * D + 32 * (tig * S::kWPT + wl);
       const unsigned char* rb = kg + (gid + 8) * 2 * D + 32 * (tig * S::kWPT + wl);
       const uint4 a0 = lds<uint4>(ra), a1 = lds<uint4>(ra + 16);
-      const uint4 b0 = lds<uint4>(rb), b1 = lds<uint4>(rb + 16);
+      uint4 b0 = make_uint4(0, 0, 0, 0), b1 = b0;
+      if constexpr (ROWS == 16) {
+        b0 = lds<uint4>(rb);
+        b1 = lds<uint4>(rb + 16);
+      }
       const uint32_t ya[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const uint32_t yb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {         // dims j = 2*q4 (+8) and 2*q4+1 (+8)
         const int st = 4 * wl + q4;
-        mma16816(s, bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x5410u)), bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x5410u)),
-                 bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x7632u)), bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)),
-                 qf[2 * st], qf[2 * st + 1]);
+        mma16816(t[st & 1], bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x5410u)),
+                 bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x5410u)), bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x7632u)),
+                 bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)), qf[2 * st], qf[2 * st + 1]);
       }
     }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) s[c] = t[0][c] + t[1][c];
   }
 
   // ------------------------------------------------------------ P . V
-  // Token-pair masks for a partial page (tokens >= nt contribute nothing).
+  // token-pair masks (tokens >= nt contribute nothing)
   __device__ __forceinline__ void pv_masks(int nt, uint32_t& m01, uint32_t& m23) {
     const int t0 = 2 * tig;
     m01 = (t0 < nt ? 0x0000FFFFu : 0u) | (t0 + 1 < nt ? 0xFFFF0000u : 0u);
@@ -537,7 +706,8 @@ struct Worker {
     }
   }
 
-  __device__ __forceinline__ void pv_fp8(const unsigned char* vg, uint32_t b0, uint32_t b1, int nt) {
+  __device__ __forceinline__ void pv_fp8(const unsigned char* vg, uint32_t b0, uint32_t b1, uint32_t lo0,
+                                         uint32_t lo1, int nt) {
     const int t0 = 2 * tig;
     constexpr int NWD = 2 * S::kUPT;          // u32 words of the thread's 8*kUPT bytes
     uint32_t x0[NWD], x1[NWD], x2[NWD], x3[NWD];
@@ -564,10 +734,13 @@ struct Worker {
       const uint32_t a2 = e4m3x2_f16(prmt(x2[ia], x3[ia], sa)) & m23;
       const uint32_t a3 = e4m3x2_f16(prmt(x2[ib], x3[ib], sb)) & m23;
       mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
+      mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
     }
   }
 
-  __device__ __forceinline__ void pv_bf16(const unsigned char* vg, uint32_t b0, uint32_t b1, int nt) {
+  template <int ROWS>
+  __device__ __forceinline__ void pv_bf16(const unsigned char* vg, uint32_t b0, uint32_t b1, uint32_t lo0,
+                                          uint32_t lo1, int nt) {
     const int t0 = 2 * tig;
     const int off = 16 * gid * S::kUPT;       // bytes of the thread's dims in a row
     uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
@@ -580,53 +753,41 @@ struct Worker {
       const uint32_t sa = (ja & 1) ? 0x7632u : 0x5410u, sb = (jb & 1) ? 0x7632u : 0x5410u;
       const uint32_t a0 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + ba), lds<uint32_t>(vg + (t0 + 1) * 2 * D + ba), sa)) & m01;
       const uint32_t a1 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + bb), lds<uint32_t>(vg + (t0 + 1) * 2 * D + bb), sb)) & m01;
-      const uint32_t a2 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa)) & m23;
-      const uint32_t a3 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb)) & m23;
+      uint32_t a2 = 0u, a3 = 0u;
+      if constexpr (ROWS == 16) {
+        a2 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa)) & m23;
+        a3 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb)) & m23;
+      }
       mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
+      mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
     }
   }
 
-  // --------------------------------------------------------- one entry
-  template <int FMT>
-  __device__ __forceinline__ void process(const unsigned char* e, const Desc& d) {
-    constexpr int CAP = FMT == KVC_FMT_TERNARY2 ? kMaxPages : (FMT == KVC_FMT_FP8_E4M3 ? 2 : 1);
-    constexpr int GB = group_bytes(FMT, D);
-    constexpr float KF = FMT == KVC_FMT_TERNARY2 ? 0.5f : 1.0f;   // ternary operands are 2c
-    const int np = d.np;
-    float s[CAP][4];
-#pragma unroll
-    for (int i = 0; i < CAP; ++i) {
-      if (i < np) {
-        if constexpr (FMT == KVC_FMT_TERNARY2) qk_ternary(e + i * GB, s[i]);
-        else if constexpr (FMT == KVC_FMT_FP8_E4M3) qk_fp8(e + i * GB, s[i]);
-        else qk_bf16(e + i * GB, s[i]);
-      }
+  // --------------------------------------------------- softmax, per page
+  // Scales the score tile, applies the row mask, moves the lazy maximum when
+  // needed, accumulates the row sums and returns P^T fragments (P scaled by
+  // the page's V scale relative to the warp's reference scale).
+  // With SPLIT, P is passed as an f16 hi + lo pair (b0/b1 and lo0/lo1,
+  // ~22 bits): pages whose values can be large (FP8, BF16) need it to keep
+  // the absolute error of P.V small; ternary values are bounded by gamma.
+  template <bool SPLIT>
+  __device__ __forceinline__ void softmax_page(float (&s)[4], float sc, float vscale, int nt, bool c0ok,
+                                               bool c1ok, uint32_t& b0, uint32_t& b1, uint32_t& lo0,
+                                               uint32_t& lo1) {
+    float x00 = s[0] * sc, x01 = s[1] * sc, x10 = s[2] * sc, x11 = s[3] * sc;
+    if (nt < kPage) {
+      if (gid >= nt) x00 = x01 = -INFINITY;
+      if (gid + 8 >= nt) x10 = x11 = -INFINITY;
     }
-    // scale, mask, entry maximum per column (cols 2*tig, 2*tig+1)
-    const bool c0ok = 2 * tig < p.G, c1ok = 2 * tig + 1 < p.G;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < CAP; ++i) {
-      if (i < np) {
-        const float sc = d.ks[i] * (KF * p.scale_log2);
-        const int nt = i == np - 1 ? d.ntok_last : kPage;
-        const bool r0 = gid < nt, r1 = gid + 8 < nt;
-        s[i][0] = (r0 && c0ok) ? s[i][0] * sc : -INFINITY;
-        s[i][1] = (r0 && c1ok) ? s[i][1] * sc : -INFINITY;
-        s[i][2] = (r1 && c0ok) ? s[i][2] * sc : -INFINITY;
-        s[i][3] = (r1 && c1ok) ? s[i][3] * sc : -INFINITY;
-        mx0 = fmaxf(mx0, fmaxf(s[i][0], s[i][2]));
-        mx1 = fmaxf(mx1, fmaxf(s[i][1], s[i][3]));
-      }
-    }
-    const bool need = mx0 > m0 + kTau || mx1 > m1 + kTau;
-    if (__any_sync(kFull, need)) {
+    const float mx0 = fmaxf(x00, x10), mx1 = fmaxf(x01, x11);
+    if (__any_sync(kFull, mx0 > m0 + kTau || mx1 > m1 + kTau)) {
+      float r0 = mx0, r1 = mx1;
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, o));
+        r0 = fmaxf(r0, __shfl_xor_sync(kFull, r0, o));
+        r1 = fmaxf(r1, __shfl_xor_sync(kFull, r1, o));
       }
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float n0 = fmaxf(m0, r0), n1 = fmaxf(m1, r1);
       const float a0 = n0 == -INFINITY ? 1.f : ex2(m0 - n0);
       const float a1 = n1 == -INFINITY ? 1.f : ex2(m1 - n1);
 #pragma unroll
@@ -639,64 +800,96 @@ struct Worker {
       m0 = n0;
       m1 = n1;
     }
-    // value-scale reference (warp-uniform: every lane reads the same desc)
-    constexpr float VF = FMT == KVC_FMT_TERNARY2 ? 0.5f : 1.0f;
-    float vmax = 0.f;
-#pragma unroll
-    for (int i = 0; i < CAP; ++i)
-      if (i < np) vmax = fmaxf(vmax, d.vs[i] * VF);
-    if (vmax > 0.f && (uref == 0.f || vmax > 16.f * uref || vmax < uref * 0.0625f)) {
-      const float beta = uref / vmax;
+    // the V scale of the page relative to the warp's reference (warp-uniform)
+    if (vscale > 0.f && (uref == 0.f || vscale > 16.f * uref || vscale < uref * 0.0625f)) {
+      const float beta = uref / vscale;
 #pragma unroll
       for (int mt = 0; mt < S::kSteps; ++mt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[mt][c] *= beta;
-      uref = vmax;
+      uref = vscale;
+      inv_uref = 1.f / vscale;
     }
-    const float inv_uref = uref > 0.f ? 1.f / uref : 0.f;
-    // P, row sums, P.V
-#pragma unroll
-    for (int i = 0; i < CAP; ++i) {
-      if (i < np) {
-        // padded GQA columns (>= G) have no finite maximum: keep them at 0
-        const float p00 = c0ok ? ex2(s[i][0] - m0) : 0.f, p01 = c1ok ? ex2(s[i][1] - m1) : 0.f;
-        const float p10 = c0ok ? ex2(s[i][2] - m0) : 0.f, p11 = c1ok ? ex2(s[i][3] - m1) : 0.f;
-        l0 += p00 + p10;
-        l1 += p01 + p11;
-        const float ratio = d.vs[i] * VF * inv_uref;
-        const uint32_t b0 = movtrans(f16x2(p00 * ratio, p01 * ratio));
-        const uint32_t b1 = movtrans(f16x2(p10 * ratio, p11 * ratio));
-        const int nt = i == np - 1 ? d.ntok_last : kPage;
-        const unsigned char* vg = e + S::kHalf + i * GB;
-        if constexpr (FMT == KVC_FMT_TERNARY2) pv_ternary(vg, b0, b1, nt);
-        else if constexpr (FMT == KVC_FMT_FP8_E4M3) pv_fp8(vg, b0, b1, nt);
-        else pv_bf16(vg, b0, b1, nt);
+    const float ratio = vscale * inv_uref;
+    const float p00 = ex2(x00 - m0), p01 = ex2(x01 - m1);
+    const float p10 = ex2(x10 - m0), p11 = ex2(x11 - m1);
+    l0 += p00 + p10;
+    l1 += p01 + p11;
+    // padded GQA columns (>= G) get P = 0
+    const float q0 = c0ok ? ratio : 0.f, q1 = c1ok ? ratio : 0.f;
+    const float y00 = p00 * q0, y01 = p01 * q1, y10 = p10 * q0, y11 = p11 * q1;
+    const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
+    b0 = movtrans(h0);
+    b1 = movtrans(h1);
+    if constexpr (SPLIT) {
+      const float2 g0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+      const float2 g1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+      lo0 = movtrans(f16x2(y00 - g0.x, y01 - g0.y));
+      lo1 = movtrans(f16x2(y10 - g1.x, y11 - g1.y));
+    }
+  }
+
+  // --------------------------------------------------------- one entry
+  __device__ __forceinline__ void process(const unsigned char* e, const Desc& d) {
+    const int fmt = d.fmt, np = d.np;
+    const bool c0ok = 2 * tig < p.G, c1ok = 2 * tig + 1 < p.G;
+    uint32_t b0, b1, lo0 = 0u, lo1 = 0u;
+    if (fmt == KVC_FMT_TERNARY2) {
+      constexpr int GB = group_bytes(KVC_FMT_TERNARY2, D);
+      for (int i = 0; i < np; ++i) {
+        const int nt = i == np - 1 ? d.nrows : kPage;
+        float s[4];
+        qk_ternary(e + i * GB, s);
+        softmax_page<false>(s, d.ks[i] * (0.5f * p.scale_log2), 0.5f * d.vs[i], nt, c0ok, c1ok, b0, b1, lo0, lo1);
+        pv_ternary(e + S::kHalf + i * GB, b0, b1, nt);
+      }
+    } else if (fmt == KVC_FMT_FP8_E4M3) {
+      constexpr int GB = group_bytes(KVC_FMT_FP8_E4M3, D);
+      for (int i = 0; i < np; ++i) {
+        const int nt = i == np - 1 ? d.nrows : kPage;
+        float s[4];
+        qk_fp8(e + i * GB, s);
+        softmax_page<true>(s, d.ks[i] * p.scale_log2, d.vs[i], nt, c0ok, c1ok, b0, b1, lo0, lo1);
+        pv_fp8(e + S::kHalf + i * GB, b0, b1, lo0, lo1, nt);
+      }
+    } else if (fmt == KVC_FMT_BF16) {
+      float s[4];
+      if constexpr (S::kBf16Rows == 16) {
+        qk_bf16<16>(e, s);
+        softmax_page<true>(s, p.scale_log2, 1.f, d.nrows, c0ok, c1ok, b0, b1, lo0, lo1);
+        pv_bf16<16>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
+      } else {
+        qk_bf16<8>(e, s);
+        softmax_page<true>(s, p.scale_log2, 1.f, d.nrows, c0ok, c1ok, b0, b1, lo0, lo1);
+        pv_bf16<8>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       }
     }
   }
 
   // ------------------------------------------------------------- main
-  __device__ void run(int w_index, int n_warps, long long units) {
+  __device__ void run(int w_index) {
     lane = threadIdx.x & 31;
     gid = lane >> 2;
     tig = lane & 3;
     W = w_index;
-    nwg = n_warps;
-    U = units;
-    u0 = (long long)W * U / nwg;
-    u1 = (long long)(W + 1) * U / nwg;
-    cursor = u0;
-    cb = u0;
-    timed_out = false;
+    const long long c0 = (long long)W * pr.C / pr.nwg, c1 = (long long)(W + 1) * pr.C / pr.nwg;
+    cursor = pr.unit_of_cost(c0);
+    u1 = pr.unit_of_cost(c1);
+    cb = cursor;
+    bf16_half = 0;
     cur_bg = -1;
-    meta_phase_a(p, pr, cb + lane, u1, cur);
-    meta_phase_b(p, cur);
-    meta_phase_a(p, pr, cb + 32 + lane, u1, nxt);
+    {
+      MetaA a;
+      meta_phase_a(p, pr, cb + lane, u1, a);
+      meta_phase_b(p, pr, a, cur);
+    }
+    meta_phase_a(p, pr, cb + 32 + lane, u1, nxa);
     nxt_b_pending = true;
 
     bool issued[kEntries];
 #pragma unroll
     for (int s = 0; s < kEntries; ++s) issued[s] = issue(s);
+    bool timed_out = false;
     for (int it = 0;; ++it) {
       const int slot = it % kEntries;
       if (!issued[slot]) break;
@@ -705,15 +898,12 @@ struct Worker {
         break;
       }
       const Desc& d = desc[slot];
-      const int fmt = d.fmt, bg = d.bg;
+      const int bg = d.bg;
       if (bg != cur_bg) {
         finish();
         begin(bg);
       }
-      const unsigned char* e = ring + slot * S::kEntryBytes;
-      if (fmt == KVC_FMT_TERNARY2) process<KVC_FMT_TERNARY2>(e, d);
-      else if (fmt == KVC_FMT_FP8_E4M3) process<KVC_FMT_FP8_E4M3>(e, d);
-      else if (fmt == KVC_FMT_BF16) process<KVC_FMT_BF16>(e, d);
+      if (d.fmt != kSkip) process(ring + slot * S::kEntryBytes, d);
       __syncwarp();
       issued[slot] = issue(slot);
     }
@@ -736,15 +926,17 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
   Desc* descs = reinterpret_cast<Desc*>(smem + kWarps * kEntries * S::kEntryBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(descs + kWarps * kEntries);
   int* seqP = reinterpret_cast<int*>(bars + kWarps * kEntries);
-  int* seqL = seqP + (p.B + 1);
+  int* seqC = seqP + (p.B + 1);
+  int* seqL = seqC + (p.B + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int whp = p.hp == KVC_FMT_BF16 ? kCostBf16 : kCostFp8;
 
   if (threadIdx.x < kWarps * kEntries) mbar_init(&bars[threadIdx.x], 1);
   if (warp == 0) {
-    int carry = 0;
+    int carry_u = 0, carry_c = 0;
     for (int base = 0; base < p.B; base += 32) {
       const int b = base + lane;
-      int u = 0;
+      int u = 0, c = 0;
       if (b < p.B) {
         int L = p.ctx[b];
         if (L < 0 || L > p.max_pages * kPage) {
@@ -752,18 +944,23 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
           L = 0;
         }
         seqL[b] = L;
-        u = ((L + kPage - 1) / kPage) * p.Hkv;
+        const SeqShape s = seq_shape(L, p.sink, p.window, whp);
+        u = s.np * p.Hkv;
+        c = s.cost * p.Hkv;
       }
-      int incl = u;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += t;
+        const int tu = __shfl_up_sync(kFull, u, o), tc = __shfl_up_sync(kFull, c, o);
+        if (lane >= o) { u += tu; c += tc; }
       }
-      if (b < p.B) seqP[b + 1] = carry + incl;
-      carry += __shfl_sync(kFull, incl, 31);
+      if (b < p.B) {
+        seqP[b + 1] = carry_u + u;
+        seqC[b + 1] = carry_c + c;
+      }
+      carry_u += __shfl_sync(kFull, u, 31);
+      carry_c += __shfl_sync(kFull, c, 31);
     }
-    if (lane == 0) seqP[0] = 0;
+    if (lane == 0) seqP[0] = seqC[0] = 0;
   }
   fence_mbar_init();
   __syncthreads();
@@ -772,38 +969,73 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
     if (seqL[b] == 0)
       for (int i = threadIdx.x; i < p.Hq * D; i += blockDim.x) p.out[(long long)b * p.Hq * D + i] = 0.f;
 
-  const long long U = seqP[p.B];
-  if (U == 0) return;
-  const int nwg = (int)((long long)p.n_splits < U ? p.n_splits : U);   // n_splits = warps in the grid
+  Prologue pr;
+  pr.seqP = seqP;
+  pr.seqC = seqC;
+  pr.seqL = seqL;
+  pr.B = p.B;
+  pr.Hkv = p.Hkv;
+  pr.sink = p.sink;
+  pr.window = p.window;
+  pr.whp = whp;
+  pr.C = seqC[p.B];
+  pr.U = seqP[p.B];
+  if (pr.U == 0) return;
+  // every worker's weight range is at least twice the heaviest unit, so
+  // each one owns at least one unit
+  const long long most = pr.C / (2 * kCostBf16);
+  pr.nwg = (int)((long long)p.n_splits < most ? p.n_splits : (most > 0 ? most : 1));
   const int W = blockIdx.x * kWarps + warp;
-  if (W >= nwg) return;
-  Worker<D> wk(p, Prologue{seqP, seqL}, ring + warp * kEntries * S::kEntryBytes, descs + warp * kEntries,
-               bars + warp * kEntries);
-  wk.run(W, nwg, U);
+  if (W >= pr.nwg) return;
+  Worker<D> wk(p, pr, ring + warp * kEntries * S::kEntryBytes, descs + warp * kEntries, bars + warp * kEntries);
+  wk.run(W);
 }
 
 template <int D>
 size_t tc_smem_bytes(int batch) {
   return (size_t)kWarps * kEntries * Shape<D>::kEntryBytes + kWarps * kEntries * sizeof(Desc) +
-         kWarps * kEntries * sizeof(uint64_t) + (size_t)(2 * batch + 1) * sizeof(int);
+         kWarps * kEntries * sizeof(uint64_t) + (size_t)(3 * batch + 2) * sizeof(int);
 }
 
+// The kernel's shared memory depends on the batch (the sequence tables); the
+// largest size is opted into once per device, and CTAs per SM are cached per
+// (device, head_dim, batch) so a call costs no runtime query after the first.
+constexpr int kMaxDev = 64;
 template <int D>
 cudaError_t tc_occupancy(int batch, int* ctas_per_sm) {
-  const size_t smem = tc_smem_bytes<D>(batch);
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static std::mutex mu;
+  static bool opted[kMaxDev] = {};
+  static std::map<std::pair<int, int>, int> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D>, kWarps * 32, smem);
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, batch);
+  const auto it = cache.find(key);
+  if (it != cache.end()) {
+    *ctas_per_sm = it->second;
+    return cudaSuccess;
+  }
+  if (dev >= 0 && dev < kMaxDev && !opted[dev]) {
+    e = cudaFuncSetAttribute(decode_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc_smem_bytes<D>(kTcMaxBatchTpl));
+    if (e != cudaSuccess) return e;
+    opted[dev] = true;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D>, kWarps * 32,
+                                                    tc_smem_bytes<D>(batch));
+  if (e == cudaSuccess) cache[key] = *ctas_per_sm;
+  return e;
 }
 
 }  // namespace
 
 // Largest batch the tensor-core kernel handles (its per-CTA sequence table
 // lives in shared memory); larger batches use the CUDA-core kernel.
-constexpr int kTcMaxBatch = 1024;
+constexpr int kTcMaxBatch = kTcMaxBatchTpl;
 
 bool tc_supported(int batch, int hkv, int max_pages) {
-  return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages < (1ll << 31);
+  return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages * kCostBf16 < (1ll << 31);
 }
 
 cudaError_t tc_grid(int batch, int d, int* grid) {
