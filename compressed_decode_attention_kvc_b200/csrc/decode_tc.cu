@@ -57,7 +57,8 @@ constexpr int kWarps = 4;            // warps per CTA; each is an independent wo
 constexpr int kEntries = 2;          // ring entries per warp
 constexpr int kMaxPages = 8;         // pages per entry
 constexpr float kTau = 8.0f;         // lazy-max threshold, log2 units
-constexpr uint32_t kSpinLimit = 1u << 22;
+constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per try
+constexpr uint32_t kSpinLimit = 4000;       // ... for at most ~4 s
 constexpr int kSkip = 3;             // entry carrying an unusable page (flagged, no data)
 constexpr unsigned kFull = 0xffffffffu;
 // Work weights of one page of one KV head, proportional to the bytes it moves.
@@ -97,14 +98,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
+// try_wait suspends the warp (it issues nothing) until the phase completes
+// or the hinted time, in ns, runs out.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs) : "memory");
   return ok != 0;
 }
-// Bounded wait: false if the phase did not complete within the limit.
+// Bounded wait: false if the phase did not complete within the limit
+// (kSpinLimit tries of at most kSuspendNs each).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t i = 0; i < kSpinLimit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -247,69 +251,168 @@ struct Prologue {
 };
 
 // ------------------------------------------------------------- metadata
-// Per-lane page metadata, packed: fmt (2 bits) | nrows (5 bits) << 2 | bg << 7.
+// Per-lane page metadata.  Phase A (block-table slot, caller tag) is loaded
+// one chunk of 32 units ahead; phase B (format, scales) once those loads
+// have landed.  Packed words keep the register footprint small:
+//   A.info: ntok (5 bits) | is_hp (1) << 5 | g (7) << 6 | bg << 13
+//   Meta.m: fmt (2 bits) | ntok (5) << 2 | bg << 7     (m < 0: no unit)
 __device__ __forceinline__ int meta_pack(int fmt, int ntok, int bg) { return fmt | (ntok << 2) | (bg << 7); }
 __device__ __forceinline__ int meta_fmt(int m) { return m & 3; }
 __device__ __forceinline__ int meta_ntok(int m) { return (m >> 2) & 31; }
 __device__ __forceinline__ int meta_bg(int m) { return m >> 7; }
 
-struct MetaA {    // after the block-table load
-  int phys, older, bg, j;   // bg < 0: no unit
+struct MetaA {
+  int phys, older, info;    // info < 0: no unit
 };
-struct Meta {     // resolved
-  int m;          // packed fmt / ntok / bg (bg = -1 encoded as m < 0)
-  int phys;
-  float ks, vs;
+struct Meta {
+  int m;                    // packed fmt / ntok / bg
+  int grp;                  // (page slot) * Hkv + g: index of the (page, head) group
+  float ks, vs;             // K / V scale of the page (gamma, s or 1)
 };
 
-__device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prologue& pr, int x, int u1,
-                                             MetaA& a) {
-  a.bg = -1;
+// Unit x -> (sequence, KV head, page) for the 32 units of a chunk starting at
+// x0.  The chunk's first unit is decoded once for the warp; lanes past the
+// end of that (sequence, KV head) decode their own unit.
+__device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prologue& pr, int x0, int u1,
+                                             int lane, MetaA& a) {
+  a.info = -1;
   a.phys = 0;
   a.older = KVC_FMT_TERNARY2;
-  a.j = 0;
+  if (x0 >= u1) return;
+  const int b0 = pr.find(pr.seqP, x0);
+  const int L0 = pr.seqL[b0];
+  const int np0 = (L0 + kPage - 1) / kPage;
+  const int off0 = x0 - pr.seqP[b0];
+  const int g0 = off0 / np0;
+  const int j0 = off0 - g0 * np0;
+  const int x = x0 + lane;
   if (x >= u1) return;
-  const int b = pr.find(pr.seqP, x);
-  const int np = (pr.seqL[b] + kPage - 1) / kPage;
-  const int off = x - pr.seqP[b];
-  const int g = off / np;
-  const int j = off - g * np;
+  int b = b0, g = g0, j = j0 + lane, L = L0;
+  if (j >= np0) {                                  // past the first (sequence, KV head)
+    b = pr.find(pr.seqP, x);
+    L = pr.seqL[b];
+    const int np = (L + kPage - 1) / kPage;
+    const int off = x - pr.seqP[b];
+    g = off / np;
+    j = off - g * np;
+  }
   const long long row = (long long)b * p.max_pages + j;
-  a.bg = b * p.Hkv + g;
-  a.j = j;
+  const int last_valid = min((j + 1) * kPage, L) - 1;
+  const int is_hp = (j * kPage < p.sink || last_valid >= L - p.window) ? 1 : 0;
+  a.info = min(kPage, L - j * kPage) | (is_hp << 5) | (g << 6) | ((b * p.Hkv + g) << 13);
   a.phys = __ldg(p.block_table + row);
   a.older = p.older_fmt ? (int)__ldg(p.older_fmt + row) : KVC_FMT_TERNARY2;
 }
 
-__device__ __forceinline__ void meta_phase_b(const DecodeParams& p, const Prologue& pr, const MetaA& a,
-                                             Meta& m) {
+__device__ __forceinline__ void meta_phase_b(const DecodeParams& p, const MetaA& a, Meta& m) {
   m.ks = m.vs = 0.f;
-  m.phys = a.phys;
-  if (a.bg < 0) {
+  m.grp = 0;
+  if (a.info < 0) {
     m.m = -1;
     return;
   }
-  const int b = a.bg / p.Hkv, g = a.bg - b * p.Hkv;
-  const int L = pr.seqL[b];
-  const int ntok = min(kPage, L - a.j * kPage);
-  int fmt = page_format(a.j, L, p.sink, p.window, p.hp, a.older);
+  const int ntok = a.info & 31, g = (a.info >> 6) & 127, bg = a.info >> 13;
+  int fmt = (a.info >> 5) & 1 ? p.hp : a.older;
   if (fmt < 0 || fmt > 2) {
     atomicOr(p.err, kErrFormat);
     fmt = kSkip;
   } else if (a.phys < 0 || a.phys >= p.cache.n_pages[fmt]) {
     atomicOr(p.err, kErrBlockTable);
     fmt = kSkip;
-  } else if (fmt == KVC_FMT_TERNARY2) {
-    m.ks = __ldg(p.cache.k_gamma + (long long)a.phys * p.Hkv + g);
-    m.vs = __ldg(p.cache.v_gamma + (long long)a.phys * p.Hkv + g);
-  } else if (fmt == KVC_FMT_FP8_E4M3) {
-    m.ks = __ldg(p.cache.k_fp8_scale + a.phys);
-    m.vs = __ldg(p.cache.v_fp8_scale + a.phys);
   } else {
-    m.ks = m.vs = 1.f;
+    m.grp = a.phys * p.Hkv + g;
+    if (fmt == KVC_FMT_TERNARY2) {
+      m.ks = __ldg(p.cache.k_gamma + m.grp);
+      m.vs = __ldg(p.cache.v_gamma + m.grp);
+    } else if (fmt == KVC_FMT_FP8_E4M3) {
+      m.ks = __ldg(p.cache.k_fp8_scale + a.phys);
+      m.vs = __ldg(p.cache.v_fp8_scale + a.phys);
+    } else {
+      m.ks = m.vs = 1.f;
+    }
   }
-  m.m = meta_pack(fmt, ntok, a.bg);
+  m.m = meta_pack(fmt, ntok, bg);
 }
+
+// Merge the partial states of one (sequence, KV head) and write its output
+// rows.  Records are read with independent loads: per-record weights
+// lane-parallel (lane k owns record k of a batch of 32), then float4 rows.
+struct MergeArgs {          // what the merge needs, passed by value
+  const float* partials;
+  float* out;
+  uint32_t* tickets;
+  int G, Hq, Hkv;
+};
+
+template <int D>
+__device__ __noinline__ void merge_partials(MergeArgs p, int bg, int w_first, int w_last, int lane) {
+  const int G = p.G;
+  const int rs = G * (D + 2);
+  const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+  const int nrec = w_last - w_first + 1;
+  // row maxima and normalisers
+  float ms[8], ls[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) { ms[r] = -INFINITY; ls[r] = 0.f; }
+  for (int k0 = 0; k0 < nrec; k0 += 32) {
+    const int k = k0 + lane;
+    const float* st = p.partials + (long long)(w_first + k + bg) * rs;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      float mk = -INFINITY;
+      if (r < G && k < nrec) mk = __ldcg(st + r * (D + 2));
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, o));
+      ms[r] = fmaxf(ms[r], mk);
+    }
+  }
+  for (int k0 = 0; k0 < nrec; k0 += 32) {
+    const int k = k0 + lane;
+    const float* st = p.partials + (long long)(w_first + k + bg) * rs;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      float lk = 0.f;
+      if (r < G && k < nrec && ms[r] != -INFINITY) lk = __ldcg(st + r * (D + 2) + 1) * ex2(__ldcg(st + r * (D + 2)) - ms[r]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
+      ls[r] += lk;
+    }
+  }
+  // output rows: lane owns D/32 consecutive dims of every row
+  constexpr int DPL = D / 32;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r >= G) break;
+    float o[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) o[i] = 0.f;
+    if (ms[r] != -INFINITY) {
+      for (int k0 = 0; k0 < nrec; k0 += 32) {
+        const int k = k0 + lane;
+        float f = 0.f;
+        if (k < nrec) f = ex2(__ldcg(p.partials + (long long)(w_first + k + bg) * rs + r * (D + 2)) - ms[r]);
+        const int kn = min(32, nrec - k0);
+#pragma unroll 4
+        for (int kk = 0; kk < kn; ++kk) {
+          const float fk = __shfl_sync(kFull, f, kk);
+          const float* row = p.partials + (long long)(w_first + k0 + kk + bg) * rs + r * (D + 2) + 2 + lane * DPL;
+#pragma unroll
+          for (int i = 0; i < DPL; i += 2) {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(row + i));
+            o[i] = fmaf(fk, v.x, o[i]);
+            o[i + 1] = fmaf(fk, v.y, o[i + 1]);
+          }
+        }
+      }
+    }
+    const float inv = ls[r] > 0.f ? 1.f / ls[r] : 0.f;
+    float* dst = p.out + ((long long)b * p.Hq + g * G + r) * D + lane * DPL;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) dst[i] = o[i] * inv;
+  }
+  if (lane == 0) p.tickets[bg] = 0u;
+}
+
 
 // ----------------------------------------------------------- the worker
 template <int D>
@@ -346,14 +449,14 @@ struct Worker {
     if (cursor >= u1) return false;
     int li = cursor - cb;
     if (li >= 32) {
-      if (nxt_b_pending) meta_phase_b(p, pr, nxa, nxt);
+      if (nxt_b_pending) meta_phase_b(p, nxa, nxt);
       cur = nxt;
       cb += 32;
       li -= 32;
-      meta_phase_a(p, pr, cb + 32 + lane, u1, nxa);
+      meta_phase_a(p, pr, cb + 32, u1, lane, nxa);
       nxt_b_pending = true;
     } else if (nxt_b_pending) {
-      meta_phase_b(p, pr, nxa, nxt);
+      meta_phase_b(p, nxa, nxt);
       nxt_b_pending = false;
     }
     const int m0l = shfl(cur.m, li);
@@ -376,13 +479,12 @@ struct Worker {
     } else {
       if (f0 != kSkip) {
         const int cap = f0 == KVC_FMT_TERNARY2 ? S::kTernCap : (f0 == KVC_FMT_FP8_E4M3 ? S::kFp8Cap : 1);
-        // only the last page of a (sequence, KV head) can be partial, and it
-        // ends the run, so every page but the entry's last is full
-        const bool ok = lane >= li && (cb + lane) < u1 && cur.m >= 0 && meta_fmt(cur.m) == f0 &&
-                        meta_bg(cur.m) == bg0;
+        // same format and (sequence, KV head); only the last page of a
+        // (sequence, KV head) can be partial, and it ends the run
+        const bool ok = lane >= li && (cb + lane) < u1 && cur.m >= 0 && ((cur.m ^ m0l) & ~(31 << 2)) == 0;
         const uint32_t run = __ballot_sync(kFull, ok) >> li;
         const int len = (run == 0xffffffffu) ? 32 : __ffs(~run) - 1;
-        np = max(1, min(len, cap));
+        np = min(len, cap);
         bytes_per_page = group_bytes(f0, D);
       }
       advance = np;
@@ -396,41 +498,34 @@ struct Worker {
       d.nrows = nrows;
       d.row0 = row0;
     }
-    if (lane >= li && lane < li + np) {
-      d.ks[lane - li] = cur.ks;
-      d.vs[lane - li] = cur.vs;
+    const int k = lane - li;
+    const bool mine = k >= 0 && k < np;
+    if (mine) {
+      d.ks[k] = cur.ks;
+      d.vs[k] = cur.vs;
     }
     __syncwarp();
     fence_proxy_async();
-    if (f0 == kSkip) {
-      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], 0);
-    } else {
-      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(2 * np * bytes_per_page));
-      __syncwarp();
-      if (lane >= li && lane < li + np) {
-        const int k = lane - li;
-        const int g = bg0 % p.Hkv;
-        const int gb = group_bytes(f0, D);
-        const long long grp = (long long)cur.phys * p.Hkv + g;
-        const unsigned char* ksrc;
-        const unsigned char* vsrc;
-        if (f0 == KVC_FMT_TERNARY2) {
-          ksrc = static_cast<const unsigned char*>(p.cache.k_tern);
-          vsrc = static_cast<const unsigned char*>(p.cache.v_tern);
-        } else if (f0 == KVC_FMT_FP8_E4M3) {
-          ksrc = static_cast<const unsigned char*>(p.cache.k_fp8);
-          vsrc = static_cast<const unsigned char*>(p.cache.v_fp8);
-        } else {
-          ksrc = static_cast<const unsigned char*>(p.cache.k_bf16);
-          vsrc = static_cast<const unsigned char*>(p.cache.v_bf16);
-        }
-        unsigned char* e = ring + slot * S::kEntryBytes;
-        bulk_g2s(e + k * bytes_per_page, ksrc + grp * gb + src_off, (uint32_t)bytes_per_page, &bars[slot]);
-        bulk_g2s(e + S::kHalf + k * bytes_per_page, vsrc + grp * gb + src_off, (uint32_t)bytes_per_page,
-                 &bars[slot]);
-      }
-    }
+    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], f0 == kSkip ? 0u : (uint32_t)(2 * np * bytes_per_page));
     __syncwarp();
+    if (f0 != kSkip && mine) {
+      const unsigned char* kb;
+      const unsigned char* vb;
+      if (f0 == KVC_FMT_TERNARY2) {
+        kb = static_cast<const unsigned char*>(p.cache.k_tern);
+        vb = static_cast<const unsigned char*>(p.cache.v_tern);
+      } else if (f0 == KVC_FMT_FP8_E4M3) {
+        kb = static_cast<const unsigned char*>(p.cache.k_fp8);
+        vb = static_cast<const unsigned char*>(p.cache.v_fp8);
+      } else {
+        kb = static_cast<const unsigned char*>(p.cache.k_bf16);
+        vb = static_cast<const unsigned char*>(p.cache.v_bf16);
+      }
+      const long long off = (long long)cur.grp * group_bytes(f0, D) + src_off;
+      unsigned char* e = ring + slot * S::kEntryBytes + k * bytes_per_page;
+      bulk_g2s(e, kb + off, (uint32_t)bytes_per_page, &bars[slot]);
+      bulk_g2s(e + S::kHalf, vb + off, (uint32_t)bytes_per_page, &bars[slot]);
+    }
     cursor += advance;
     return true;
   }
@@ -512,78 +607,7 @@ struct Worker {
     last = __shfl_sync(kFull, last, 0);
     if (!last) return;
     __threadfence();
-    merge(bg, w_first, w_last);
-  }
-
-  // Merge the partial states of one (sequence, KV head) and write its output
-  // rows.  Records are read with independent loads: per-record weights
-  // lane-parallel (lane k owns record k of a batch of 32), then float4 rows.
-  __device__ void merge(int bg, int w_first, int w_last) {
-    const int G = p.G;
-    const int rs = G * (D + 2);
-    const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-    const int nrec = w_last - w_first + 1;
-    // row maxima and normalisers
-    float ms[8], ls[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) { ms[r] = -INFINITY; ls[r] = 0.f; }
-    for (int k0 = 0; k0 < nrec; k0 += 32) {
-      const int k = k0 + lane;
-      const float* st = p.partials + (long long)(w_first + k + bg) * rs;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        float mk = -INFINITY;
-        if (r < G && k < nrec) mk = __ldcg(st + r * (D + 2));
-#pragma unroll
-        for (int o = 16; o; o >>= 1) mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, o));
-        ms[r] = fmaxf(ms[r], mk);
-      }
-    }
-    for (int k0 = 0; k0 < nrec; k0 += 32) {
-      const int k = k0 + lane;
-      const float* st = p.partials + (long long)(w_first + k + bg) * rs;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        float lk = 0.f;
-        if (r < G && k < nrec && ms[r] != -INFINITY) lk = __ldcg(st + r * (D + 2) + 1) * ex2(__ldcg(st + r * (D + 2)) - ms[r]);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) lk += __shfl_xor_sync(kFull, lk, o);
-        ls[r] += lk;
-      }
-    }
-    // output rows: lane owns D/32 consecutive dims of every row
-    constexpr int DPL = D / 32;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (r >= G) break;
-      float o[DPL];
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) o[i] = 0.f;
-      if (ms[r] != -INFINITY) {
-        for (int k0 = 0; k0 < nrec; k0 += 32) {
-          const int k = k0 + lane;
-          float f = 0.f;
-          if (k < nrec) f = ex2(__ldcg(p.partials + (long long)(w_first + k + bg) * rs + r * (D + 2)) - ms[r]);
-          const int kn = min(32, nrec - k0);
-#pragma unroll 4
-          for (int kk = 0; kk < kn; ++kk) {
-            const float fk = __shfl_sync(kFull, f, kk);
-            const float* row = p.partials + (long long)(w_first + k0 + kk + bg) * rs + r * (D + 2) + 2 + lane * DPL;
-#pragma unroll
-            for (int i = 0; i < DPL; i += 2) {
-              const float2 v = __ldcg(reinterpret_cast<const float2*>(row + i));
-              o[i] = fmaf(fk, v.x, o[i]);
-              o[i + 1] = fmaf(fk, v.y, o[i + 1]);
-            }
-          }
-        }
-      }
-      const float inv = ls[r] > 0.f ? 1.f / ls[r] : 0.f;
-      float* dst = p.out + ((long long)b * p.Hq + g * G + r) * D + lane * DPL;
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) dst[i] = o[i] * inv;
-    }
-    if (lane == 0) p.tickets[bg] = 0u;
+    merge_partials<D>(MergeArgs{p.partials, p.out, p.tickets, p.G, p.Hq, p.Hkv}, bg, w_first, w_last, lane);
   }
 
   // ---------------------------------------------------------- Q . K^T
@@ -771,15 +795,19 @@ struct Worker {
   // ~22 bits): pages whose values can be large (FP8, BF16) need it to keep
   // the absolute error of P.V small; ternary values are bounded by gamma.
   template <bool SPLIT>
-  __device__ __forceinline__ void softmax_page(float (&s)[4], float sc, float vscale, int nt, bool c0ok,
-                                               bool c1ok, uint32_t& b0, uint32_t& b1, uint32_t& lo0,
+  __device__ __forceinline__ void softmax_page(float (&s)[4], float sc, float ratio, int nt, float c0f,
+                                               float c1f, uint32_t& b0, uint32_t& b1, uint32_t& lo0,
                                                uint32_t& lo1) {
-    float x00 = s[0] * sc, x01 = s[1] * sc, x10 = s[2] * sc, x11 = s[3] * sc;
+    // exponent arguments s*sc - m; the scale sc is >= 0 (gamma, s or 1)
+    float mx0 = fmaxf(s[0], s[2]) * sc, mx1 = fmaxf(s[1], s[3]) * sc;
+    bool masked = false;
     if (nt < kPage) {
-      if (gid >= nt) x00 = x01 = -INFINITY;
-      if (gid + 8 >= nt) x10 = x11 = -INFINITY;
+      masked = true;
+      const bool r0 = gid < nt, r1 = gid + 8 < nt;
+      mx0 = r1 ? mx0 : s[0] * sc;
+      mx1 = r1 ? mx1 : s[1] * sc;
+      if (!r0) mx0 = mx1 = -INFINITY;
     }
-    const float mx0 = fmaxf(x00, x10), mx1 = fmaxf(x01, x11);
     if (__any_sync(kFull, mx0 > m0 + kTau || mx1 > m1 + kTau)) {
       float r0 = mx0, r1 = mx1;
 #pragma unroll
@@ -800,23 +828,18 @@ struct Worker {
       m0 = n0;
       m1 = n1;
     }
-    // the V scale of the page relative to the warp's reference (warp-uniform)
-    if (vscale > 0.f && (uref == 0.f || vscale > 16.f * uref || vscale < uref * 0.0625f)) {
-      const float beta = uref / vscale;
-#pragma unroll
-      for (int mt = 0; mt < S::kSteps; ++mt)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[mt][c] *= beta;
-      uref = vscale;
-      inv_uref = 1.f / vscale;
+    float e00 = fmaf(s[0], sc, -m0), e01 = fmaf(s[1], sc, -m1);
+    float e10 = fmaf(s[2], sc, -m0), e11 = fmaf(s[3], sc, -m1);
+    if (masked) {
+      if (gid >= nt) e00 = e01 = -INFINITY;
+      if (gid + 8 >= nt) e10 = e11 = -INFINITY;
     }
-    const float ratio = vscale * inv_uref;
-    const float p00 = ex2(x00 - m0), p01 = ex2(x01 - m1);
-    const float p10 = ex2(x10 - m0), p11 = ex2(x11 - m1);
+    const float p00 = ex2(e00), p01 = ex2(e01), p10 = ex2(e10), p11 = ex2(e11);
     l0 += p00 + p10;
     l1 += p01 + p11;
-    // padded GQA columns (>= G) get P = 0
-    const float q0 = c0ok ? ratio : 0.f, q1 = c1ok ? ratio : 0.f;
+    // P scaled by the page's V scale (relative to the reference); padded GQA
+    // columns (>= G) get P = 0
+    const float q0 = c0f * ratio, q1 = c1f * ratio;
     const float y00 = p00 * q0, y01 = p01 * q1, y10 = p10 * q0, y11 = p11 * q1;
     const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
     b0 = movtrans(h0);
@@ -829,44 +852,82 @@ struct Worker {
     }
   }
 
+  // Re-base the warp's value-scale reference when the entry's V scales
+  // (vf * vs[i]) leave [ref/16, 16*ref]: P = p * vs / ref stays well inside
+  // the f16 normal range.  Warp-uniform (every lane reads the same desc).
+  __device__ __forceinline__ void rebase_value_scale(const Desc& d, float vf) {
+    float vmax = 0.f, vmin = INFINITY;
+    for (int i = 0; i < d.np; ++i) {
+      const float v = d.vs[i] * vf;
+      vmax = fmaxf(vmax, v);
+      vmin = fminf(vmin, v);
+    }
+    if (vmax > 0.f && (uref == 0.f || vmax > 16.f * uref || vmin < uref * 0.0625f)) {
+      const float beta = uref / vmax;
+#pragma unroll
+      for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[mt][c] *= beta;
+      uref = vmax;
+      inv_uref = 1.f / vmax;
+    }
+  }
+
   // --------------------------------------------------------- one entry
   __device__ __forceinline__ void process(const unsigned char* e, const Desc& d) {
     const int fmt = d.fmt, np = d.np;
-    const bool c0ok = 2 * tig < p.G, c1ok = 2 * tig + 1 < p.G;
+    const float c0f = 2 * tig < p.G ? 1.f : 0.f, c1f = 2 * tig + 1 < p.G ? 1.f : 0.f;
     uint32_t b0, b1, lo0 = 0u, lo1 = 0u;
     if (fmt == KVC_FMT_TERNARY2) {
       constexpr int GB = group_bytes(KVC_FMT_TERNARY2, D);
+      rebase_value_scale(d, 0.5f);
+      const float kf = 0.5f * p.scale_log2, vf = 0.5f * inv_uref;
       for (int i = 0; i < np; ++i) {
         const int nt = i == np - 1 ? d.nrows : kPage;
         float s[4];
         qk_ternary(e + i * GB, s);
-        softmax_page<false>(s, d.ks[i] * (0.5f * p.scale_log2), 0.5f * d.vs[i], nt, c0ok, c1ok, b0, b1, lo0, lo1);
+        softmax_page<false>(s, d.ks[i] * kf, d.vs[i] * vf, nt, c0f, c1f, b0, b1, lo0, lo1);
         pv_ternary(e + S::kHalf + i * GB, b0, b1, nt);
       }
     } else if (fmt == KVC_FMT_FP8_E4M3) {
       constexpr int GB = group_bytes(KVC_FMT_FP8_E4M3, D);
+      rebase_value_scale(d, 1.f);
       for (int i = 0; i < np; ++i) {
         const int nt = i == np - 1 ? d.nrows : kPage;
         float s[4];
         qk_fp8(e + i * GB, s);
-        softmax_page<true>(s, d.ks[i] * p.scale_log2, d.vs[i], nt, c0ok, c1ok, b0, b1, lo0, lo1);
+        softmax_page<true>(s, d.ks[i] * p.scale_log2, d.vs[i] * inv_uref, nt, c0f, c1f, b0, b1, lo0, lo1);
         pv_fp8(e + S::kHalf + i * GB, b0, b1, lo0, lo1, nt);
       }
     } else if (fmt == KVC_FMT_BF16) {
+      rebase_value_scale(d, 1.f);
       float s[4];
       if constexpr (S::kBf16Rows == 16) {
         qk_bf16<16>(e, s);
-        softmax_page<true>(s, p.scale_log2, 1.f, d.nrows, c0ok, c1ok, b0, b1, lo0, lo1);
+        softmax_page<true>(s, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
         pv_bf16<16>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       } else {
         qk_bf16<8>(e, s);
-        softmax_page<true>(s, p.scale_log2, 1.f, d.nrows, c0ok, c1ok, b0, b1, lo0, lo1);
+        softmax_page<true>(s, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
         pv_bf16<8>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       }
     }
   }
 
   // ------------------------------------------------------------- main
+  __device__ __forceinline__ bool consume(int slot, uint32_t parity) {
+    if (!mbar_wait(&bars[slot], parity)) return false;
+    const Desc& d = desc[slot];
+    const int bg = d.bg;
+    if (bg != cur_bg) {
+      finish();
+      begin(bg);
+    }
+    if (d.fmt != kSkip) process(ring + slot * S::kEntryBytes, d);
+    __syncwarp();
+    return true;
+  }
+
   __device__ void run(int w_index) {
     lane = threadIdx.x & 31;
     gid = lane >> 2;
@@ -880,38 +941,26 @@ struct Worker {
     cur_bg = -1;
     {
       MetaA a;
-      meta_phase_a(p, pr, cb + lane, u1, a);
-      meta_phase_b(p, pr, a, cur);
+      meta_phase_a(p, pr, cb, u1, lane, a);
+      meta_phase_b(p, a, cur);
     }
-    meta_phase_a(p, pr, cb + 32 + lane, u1, nxa);
+    meta_phase_a(p, pr, cb + 32, u1, lane, nxa);
     nxt_b_pending = true;
 
-    bool issued[kEntries];
-#pragma unroll
-    for (int s = 0; s < kEntries; ++s) issued[s] = issue(s);
-    bool timed_out = false;
-    for (int it = 0;; ++it) {
-      const int slot = it % kEntries;
-      if (!issued[slot]) break;
-      if (!mbar_wait(&bars[slot], (uint32_t)((it / kEntries) & 1))) {
-        timed_out = true;
-        break;
-      }
-      const Desc& d = desc[slot];
-      const int bg = d.bg;
-      if (bg != cur_bg) {
-        finish();
-        begin(bg);
-      }
-      if (d.fmt != kSkip) process(ring + slot * S::kEntryBytes, d);
-      __syncwarp();
-      issued[slot] = issue(slot);
+    bool v0 = issue(0), v1 = issue(1);
+    bool ok = true;
+    for (int it = 0;; ++it) {          // one call site: the hot loop stays compact
+      const int slot = it & 1;
+      if (!(slot ? v1 : v0)) break;
+      if (!(ok = consume(slot, (uint32_t)(it >> 1) & 1u))) break;
+      const bool nv = issue(slot);
+      if (slot) v1 = nv; else v0 = nv;
     }
-    if (timed_out) {
+    if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrTimeout);
       // let copies still in flight land before the CTA's memory is released
-      for (int s = 0; s < kEntries; ++s)
-        if (issued[s]) mbar_wait(&bars[s], 0u), mbar_wait(&bars[s], 1u);
+      mbar_wait(&bars[0], 0u), mbar_wait(&bars[0], 1u);
+      mbar_wait(&bars[1], 0u), mbar_wait(&bars[1], 1u);
       return;
     }
     finish();
