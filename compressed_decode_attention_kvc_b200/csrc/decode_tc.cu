@@ -882,13 +882,22 @@ struct Worker {
       constexpr int GB = group_bytes(KVC_FMT_TERNARY2, D);
       rebase_value_scale(d, 0.5f);
       const float kf = 0.5f * p.scale_log2, vf = 0.5f * inv_uref;
-      for (int i = 0; i < np; ++i) {
-        const int nt = i == np - 1 ? d.nrows : kPage;
-        float s[4];
-        qk_ternary(e + i * GB, s);
-        softmax_page<false>(s, d.ks[i] * kf, d.vs[i] * vf, nt, c0f, c1f, b0, b1, lo0, lo1);
-        pv_ternary(e + S::kHalf + i * GB, b0, b1, nt);
+      // software pipeline: the scores of page i+1 are computed while page i
+      // goes through the softmax and P.V (independent instruction streams);
+      // only the entry's last page can be partial
+      float s[4];
+      qk_ternary(e, s);
+      int i = 0;
+      for (; i + 1 < np; ++i) {
+        float sn[4];
+        qk_ternary(e + (i + 1) * GB, sn);
+        softmax_page<false>(s, d.ks[i] * kf, d.vs[i] * vf, kPage, c0f, c1f, b0, b1, lo0, lo1);
+        pv_ternary(e + S::kHalf + i * GB, b0, b1, kPage);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) s[c] = sn[c];
       }
+      softmax_page<false>(s, d.ks[i] * kf, d.vs[i] * vf, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+      pv_ternary(e + S::kHalf + i * GB, b0, b1, d.nrows);
     } else if (fmt == KVC_FMT_FP8_E4M3) {
       constexpr int GB = group_bytes(KVC_FMT_FP8_E4M3, D);
       rebase_value_scale(d, 1.f);
