@@ -76,11 +76,14 @@ struct Shape {
   static constexpr int kHalf = kEntryBytes / 2;            // K region | V region
   static constexpr int kSteps = D / 16;                    // k-steps of Q.K^T = m-tiles of P.V
   static constexpr int kWPT = D / 64;                      // K words (16 dims) per thread per token
+  static constexpr int kQ8 = 4 * kWPT;                     // int8 Q fragments (hi or lo) per thread
   static constexpr int kUPT = D / 64;                      // V units (8 dims) per thread
   static constexpr int kVW = kUPT > 1 ? kUPT / 2 : 1;      // V code words per thread per token
   static constexpr int kTernCap = kHalf / (4 * D) < kMaxPages ? kHalf / (4 * D) : kMaxPages;
   static constexpr int kFp8Cap = kHalf / (16 * D);
   static constexpr int kBf16Rows = kHalf / (2 * D) >= 16 ? 16 : 8;   // token rows of a BF16 page per entry
+  static constexpr int kQBytes = 2 * kSteps * 32 * 4;      // per-warp f16 Q fragments
+  static_assert(kTernCap >= 1 && kFp8Cap >= 1 && kHalf >= 8 * 2 * D, "an entry must hold one page of each format");
 };
 
 __host__ __device__ constexpr int group_bytes(int fmt, int d) {
@@ -127,15 +130,22 @@ __device__ __forceinline__ void fence_mbar_init() {
 }
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// int8 x int8 -> int32, m16n8k32: four 8-bit k-elements per register
+__device__ __forceinline__ void imma16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ uint32_t movtrans(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 __device__ __forceinline__ float ex2(float x) {
@@ -155,6 +165,12 @@ __device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
 // pair of 2*code: 01 -> 0x4000 (+2), 11 -> 0xC000 (-2), 00 -> 0 (10 -> -0).
 __device__ __forceinline__ uint32_t tern2(uint32_t w, int o) {
   return (o == 14 ? w : (w << (14 - o))) & 0xC000C000u;
+}
+// Ternary field f (0..3) of each byte of w -> four int8 of 64*code: the
+// 2-bit field moved to bits 6..7 of its byte is 01 -> 64, 11 -> -64, 00 -> 0
+// (10 -> -128).  One AND (and one shift for f < 3) per four codes.
+__device__ __forceinline__ uint32_t tern8(uint32_t w, int f) {
+  return (f == 3 ? w : (w << (6 - 2 * f))) & 0xC0C0C0C0u;
 }
 // Two e4m3 bytes (low byte -> low half) -> f16x2.
 __device__ __forceinline__ uint32_t e4m3x2_f16(uint32_t two_bytes) {
@@ -421,6 +437,7 @@ struct Worker {
   const DecodeParams& p;
   const Prologue& pr;
   unsigned char* ring;     // this warp's kEntries entries
+  uint32_t* qsm;           // this warp's f16 Q fragments: [kSteps / 2][32 lanes][4]
   Desc* desc;              // [kEntries]
   uint64_t* bars;          // [kEntries]
   int lane, gid, tig;
@@ -433,12 +450,16 @@ struct Worker {
 
   // per (sequence, KV head) state
   int cur_bg;
-  uint32_t qf[2 * S::kSteps];
+  // Q of the group as int8 hi/lo fragments for ternary pages:
+  // q ~= sq * (128 * hi + lo), sq = max|q| / 16256 per query head
+  uint32_t qh[S::kQ8], ql[S::kQ8];
+  float kq0, kq1;          // score scale of the thread's two columns: sq * log2(e) * softmax_scale / 64
   float acc[S::kSteps][4];
   float m0, m1, l0, l1, uref, inv_uref;
 
-  __device__ Worker(const DecodeParams& pp, const Prologue& prr, unsigned char* r, Desc* d, uint64_t* b)
-      : p(pp), pr(prr), ring(r), desc(d), bars(b) {}
+  __device__ Worker(const DecodeParams& pp, const Prologue& prr, unsigned char* r, uint32_t* q, Desc* d,
+                    uint64_t* b)
+      : p(pp), pr(prr), ring(r), qsm(q), desc(d), bars(b) {}
 
   __device__ __forceinline__ int shfl(int v, int src) { return __shfl_sync(kFull, v, src); }
   __device__ __forceinline__ float shflf(float v, int src) { return __shfl_sync(kFull, v, src); }
@@ -548,13 +569,46 @@ struct Worker {
 #pragma unroll
       for (int i = 0; i < S::kWPT * 8; ++i) raw[i] = 0u;
     }
-    // qf[ri] = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) + (ri & 7) (thread-local dims)
+    // f16 B fragments for FP8 / BF16 pages, kept in shared memory:
+    // fragment ri = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) + (ri & 7)
+    // (thread-local dims), stored at [ri >> 2][lane][ri & 3]
 #pragma unroll
     for (int ri = 0; ri < 2 * S::kSteps; ++ri) {
       const int wl = ri >> 3, j = ri & 7;
       const uint32_t wa = raw[8 * wl + (j >> 1)], wb = raw[8 * wl + 4 + (j >> 1)];
-      qf[ri] = bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
+      qsm[((ri >> 2) * 32 + lane) * 4 + (ri & 3)] = bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
     }
+    // int8 hi/lo B fragments for ternary pages.  Fragment j carries, in
+    // byte i, the thread-local dim 16 * (j >> 2) + 4 * i + (j & 3): the dims
+    // whose codes tern8(word j >> 2, j & 3) puts in the same byte slots.
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < S::kWPT * 8; ++i)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(raw[i] << 16)), fabsf(__uint_as_float(raw[i] & 0xFFFF0000u))));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+    const float inv = amax > 0.f ? 16256.f / amax : 0.f;
+#pragma unroll
+    for (int j = 0; j < S::kQ8; ++j) {
+      uint32_t h = 0u, l = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int ld = 16 * (j >> 2) + 4 * i + (j & 3);
+        const uint32_t w = raw[ld >> 1];
+        const float x = __uint_as_float((ld & 1) ? (w & 0xFFFF0000u) : (w << 16));
+        const int qi = __float2int_rn(x * inv);      // |qi| <= 16256
+        const int hi = (qi + 64) >> 7;               // -127..127
+        const int lo = qi - (hi << 7);               // -64..63
+        h |= (uint32_t)(hi & 0xFF) << (8 * i);
+        l |= (uint32_t)(lo & 0xFF) << (8 * i);
+      }
+      qh[j] = h;
+      ql[j] = l;
+    }
+    const float sq = amax * (1.f / 16256.f);
+    const float f = p.scale_log2 * (1.f / 64.f);
+    kq0 = __shfl_sync(kFull, sq, 8 * tig) * f;          // head 2 * tig (lane group gid = 2 * tig)
+    kq1 = __shfl_sync(kFull, sq, 8 * tig + 4) * f;      // head 2 * tig + 1
 #pragma unroll
     for (int mt = 0; mt < S::kSteps; ++mt)
 #pragma unroll
@@ -611,7 +665,9 @@ struct Worker {
   }
 
   // ---------------------------------------------------------- Q . K^T
-  // two independent accumulation chains, summed at the end
+  // Ternary page: int8 tensor-core products of the codes (64 * c) with the
+  // hi and lo parts of Q; the two int32 chains combine exactly to
+  // 64 * sum_d c_d * q_int_d.
   __device__ __forceinline__ void qk_ternary(const unsigned char* kg, float (&s)[4]) {
     uint32_t wa[S::kWPT], wb[S::kWPT];
     const unsigned char* ra = kg + gid * (D / 4) + 4 * tig * S::kWPT;
@@ -626,16 +682,22 @@ struct Worker {
       wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
       wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
     }
-    float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    int th[4] = {0, 0, 0, 0}, tl[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int st = 0; st < S::kSteps; ++st) {
-      const int r0 = 2 * st, r1 = 2 * st + 1;
-      const int w0 = r0 >> 3, o0 = 2 * (r0 & 7), w1 = r1 >> 3, o1 = 2 * (r1 & 7);
-      mma16816(t[st & 1], tern2(wa[w0], o0), tern2(wb[w0], o0), tern2(wa[w1], o1), tern2(wb[w1], o1),
-               qf[r0], qf[r1]);
+    for (int st = 0; st < S::kQ8 / 2; ++st) {
+      const int j0 = 2 * st, j1 = 2 * st + 1;
+      const uint32_t a0 = tern8(wa[j0 >> 2], j0 & 3), a1 = tern8(wb[j0 >> 2], j0 & 3);
+      const uint32_t a2 = tern8(wa[j1 >> 2], j1 & 3), a3 = tern8(wb[j1 >> 2], j1 & 3);
+      imma16832(th, a0, a1, a2, a3, qh[j0], qh[j1]);
+      imma16832(tl, a0, a1, a2, a3, ql[j0], ql[j1]);
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) s[c] = t[0][c] + t[1][c];
+    for (int c = 0; c < 4; ++c) s[c] = (float)(th[c] * 128 + tl[c]);
+  }
+
+  // f16 Q fragments of k-steps 2k and 2k + 1
+  __device__ __forceinline__ uint4 qfrag(int k) const {
+    return *reinterpret_cast<const uint4*>(qsm + (k * 32 + lane) * 4);
   }
 
   __device__ __forceinline__ void qk_fp8(const unsigned char* kg, float (&s)[4]) {
@@ -651,8 +713,9 @@ struct Worker {
         const uint32_t pa = prmt(j < 4 ? xa.x : xa.y, j < 4 ? xa.z : xa.w, sel);
         const uint32_t pb = prmt(j < 4 ? xb.x : xb.y, j < 4 ? xb.z : xb.w, sel);
         const int st = 4 * wl + q4;
+        const uint4 qv = qfrag(st >> 1);
         mma16816(t[st & 1], e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16),
-                 qf[2 * st], qf[2 * st + 1]);
+                 (st & 1) ? qv.z : qv.x, (st & 1) ? qv.w : qv.y);
       }
     }
 #pragma unroll
@@ -678,9 +741,10 @@ struct Worker {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {         // dims j = 2*q4 (+8) and 2*q4+1 (+8)
         const int st = 4 * wl + q4;
+        const uint4 qv = qfrag(st >> 1);
         mma16816(t[st & 1], bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x5410u)),
                  bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x5410u)), bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x7632u)),
-                 bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)), qf[2 * st], qf[2 * st + 1]);
+                 bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)), (st & 1) ? qv.z : qv.x, (st & 1) ? qv.w : qv.y);
       }
     }
 #pragma unroll
@@ -795,17 +859,18 @@ struct Worker {
   // ~22 bits): pages whose values can be large (FP8, BF16) need it to keep
   // the absolute error of P.V small; ternary values are bounded by gamma.
   template <bool SPLIT>
-  __device__ __forceinline__ void softmax_page(float (&s)[4], float sc, float ratio, int nt, float c0f,
-                                               float c1f, uint32_t& b0, uint32_t& b1, uint32_t& lo0,
+  // sc0 / sc1 scale the thread's two score columns (s[0], s[2] and s[1], s[3]).
+  __device__ __forceinline__ void softmax_page(float (&s)[4], float sc0, float sc1, float ratio, int nt,
+                                               float c0f, float c1f, uint32_t& b0, uint32_t& b1, uint32_t& lo0,
                                                uint32_t& lo1) {
-    // exponent arguments s*sc - m; the scale sc is >= 0 (gamma, s or 1)
-    float mx0 = fmaxf(s[0], s[2]) * sc, mx1 = fmaxf(s[1], s[3]) * sc;
+    // exponent arguments s*sc - m; the scales are >= 0 (gamma, s or 1, times max|q|)
+    float mx0 = fmaxf(s[0], s[2]) * sc0, mx1 = fmaxf(s[1], s[3]) * sc1;
     bool masked = false;
     if (nt < kPage) {
       masked = true;
       const bool r0 = gid < nt, r1 = gid + 8 < nt;
-      mx0 = r1 ? mx0 : s[0] * sc;
-      mx1 = r1 ? mx1 : s[1] * sc;
+      mx0 = r1 ? mx0 : s[0] * sc0;
+      mx1 = r1 ? mx1 : s[1] * sc1;
       if (!r0) mx0 = mx1 = -INFINITY;
     }
     if (__any_sync(kFull, mx0 > m0 + kTau || mx1 > m1 + kTau)) {
@@ -828,8 +893,8 @@ struct Worker {
       m0 = n0;
       m1 = n1;
     }
-    float e00 = fmaf(s[0], sc, -m0), e01 = fmaf(s[1], sc, -m1);
-    float e10 = fmaf(s[2], sc, -m0), e11 = fmaf(s[3], sc, -m1);
+    float e00 = fmaf(s[0], sc0, -m0), e01 = fmaf(s[1], sc1, -m1);
+    float e10 = fmaf(s[2], sc0, -m0), e11 = fmaf(s[3], sc1, -m1);
     if (masked) {
       if (gid >= nt) e00 = e01 = -INFINITY;
       if (gid + 8 >= nt) e10 = e11 = -INFINITY;
@@ -881,7 +946,7 @@ struct Worker {
     if (fmt == KVC_FMT_TERNARY2) {
       constexpr int GB = group_bytes(KVC_FMT_TERNARY2, D);
       rebase_value_scale(d, 0.5f);
-      const float kf = 0.5f * p.scale_log2, vf = 0.5f * inv_uref;
+      const float vf = 0.5f * inv_uref;
       // software pipeline: the scores of page i+1 are computed while page i
       // goes through the softmax and P.V (independent instruction streams);
       // only the entry's last page can be partial
@@ -891,12 +956,12 @@ struct Worker {
       for (; i + 1 < np; ++i) {
         float sn[4];
         qk_ternary(e + (i + 1) * GB, sn);
-        softmax_page<false>(s, d.ks[i] * kf, d.vs[i] * vf, kPage, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<false>(s, d.ks[i] * kq0, d.ks[i] * kq1, d.vs[i] * vf, kPage, c0f, c1f, b0, b1, lo0, lo1);
         pv_ternary(e + S::kHalf + i * GB, b0, b1, kPage);
 #pragma unroll
         for (int c = 0; c < 4; ++c) s[c] = sn[c];
       }
-      softmax_page<false>(s, d.ks[i] * kf, d.vs[i] * vf, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+      softmax_page<false>(s, d.ks[i] * kq0, d.ks[i] * kq1, d.vs[i] * vf, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
       pv_ternary(e + S::kHalf + i * GB, b0, b1, d.nrows);
     } else if (fmt == KVC_FMT_FP8_E4M3) {
       constexpr int GB = group_bytes(KVC_FMT_FP8_E4M3, D);
@@ -905,7 +970,8 @@ struct Worker {
         const int nt = i == np - 1 ? d.nrows : kPage;
         float s[4];
         qk_fp8(e + i * GB, s);
-        softmax_page<true>(s, d.ks[i] * p.scale_log2, d.vs[i] * inv_uref, nt, c0f, c1f, b0, b1, lo0, lo1);
+        const float sc = d.ks[i] * p.scale_log2;
+        softmax_page<true>(s, sc, sc, d.vs[i] * inv_uref, nt, c0f, c1f, b0, b1, lo0, lo1);
         pv_fp8(e + S::kHalf + i * GB, b0, b1, lo0, lo1, nt);
       }
     } else if (fmt == KVC_FMT_BF16) {
@@ -913,11 +979,11 @@ struct Worker {
       float s[4];
       if constexpr (S::kBf16Rows == 16) {
         qk_bf16<16>(e, s);
-        softmax_page<true>(s, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
         pv_bf16<16>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       } else {
         qk_bf16<8>(e, s);
-        softmax_page<true>(s, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
         pv_bf16<8>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       }
     }
@@ -981,7 +1047,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
   using S = Shape<D>;
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* ring = smem;
-  Desc* descs = reinterpret_cast<Desc*>(smem + kWarps * kEntries * S::kEntryBytes);
+  uint32_t* qbuf = reinterpret_cast<uint32_t*>(smem + kWarps * kEntries * S::kEntryBytes);
+  Desc* descs = reinterpret_cast<Desc*>(smem + kWarps * kEntries * S::kEntryBytes + kWarps * S::kQBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(descs + kWarps * kEntries);
   int* seqP = reinterpret_cast<int*>(bars + kWarps * kEntries);
   int* seqC = seqP + (p.B + 1);
@@ -1045,13 +1112,15 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
   pr.nwg = (int)((long long)p.n_splits < most ? p.n_splits : (most > 0 ? most : 1));
   const int W = blockIdx.x * kWarps + warp;
   if (W >= pr.nwg) return;
-  Worker<D> wk(p, pr, ring + warp * kEntries * S::kEntryBytes, descs + warp * kEntries, bars + warp * kEntries);
+  Worker<D> wk(p, pr, ring + warp * kEntries * S::kEntryBytes, qbuf + warp * (S::kQBytes / 4),
+               descs + warp * kEntries, bars + warp * kEntries);
   wk.run(W);
 }
 
 template <int D>
 size_t tc_smem_bytes(int batch) {
-  return (size_t)kWarps * kEntries * Shape<D>::kEntryBytes + kWarps * kEntries * sizeof(Desc) +
+  return (size_t)kWarps * kEntries * Shape<D>::kEntryBytes + (size_t)kWarps * Shape<D>::kQBytes +
+         kWarps * kEntries * sizeof(Desc) +
          kWarps * kEntries * sizeof(uint64_t) + (size_t)(3 * batch + 2) * sizeof(int);
 }
 
