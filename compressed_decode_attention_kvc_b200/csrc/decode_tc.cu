@@ -53,7 +53,6 @@ namespace {
 
 constexpr int kTcMaxBatchTpl = 1024;   // largest batch of the tensor-core kernel
 
-constexpr int kWarps = 4;            // warps per CTA; each is an independent worker
 constexpr int kEntries = 2;          // ring entries per warp
 constexpr int kMaxPages = 8;         // pages per entry
 constexpr float kTau = 8.0f;         // lazy-max threshold, log2 units
@@ -61,8 +60,13 @@ constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per try
 constexpr uint32_t kSpinLimit = 4000;       // ... for at most ~4 s
 constexpr int kSkip = 3;             // entry carrying an unusable page (flagged, no data)
 constexpr unsigned kFull = 0xffffffffu;
-// Work weights of one page of one KV head, proportional to the bytes it moves.
-constexpr int kCostTern = 1, kCostFp8 = 4, kCostBf16 = 8;
+// Work weights of one page of one KV head: the warp time it costs relative to
+// a ternary page (measured on B200: unpacking and the per-entry issue work
+// make a page's time grow more slowly than its bytes).  kCostBf16 is the
+// largest weight (it bounds the weight arithmetic).
+constexpr int kCostTern = 1, kCostFp8 = 4, kCostBf16 = 7;
+template <int D>
+__host__ __device__ constexpr int cost_bf16() { return D == 256 ? 7 : 6; }
 
 struct Desc {
   int fmt, np, bg, nrows;            // nrows: valid token rows of the entry's last page
@@ -70,20 +74,24 @@ struct Desc {
   float ks[kMaxPages], vs[kMaxPages];
 };
 
-template <int D>
+// HPC: KV heads per CTA (1, 2 or 4), one warp each.  The warps of a CTA walk
+// the same pages; a ring slot holds those pages for all HPC heads.
+template <int D, int HPC>
 struct Shape {
-  static constexpr int kEntryBytes = D == 64 ? 4096 : 8192;
-  static constexpr int kHalf = kEntryBytes / 2;            // K region | V region
+  static constexpr int kEntryBytes = D == 64 ? 4096 : 8192;   // per head
+  static constexpr int kHeadHalf = kEntryBytes / 2;         // K (or V) bytes of one head per slot
+  static constexpr int kSlotBytes = HPC * kEntryBytes;      // one ring slot of the CTA
+  static constexpr int kHalf = kSlotBytes / 2;              // K region | V region
   static constexpr int kSteps = D / 16;                    // k-steps of Q.K^T = m-tiles of P.V
   static constexpr int kWPT = D / 64;                      // K words (16 dims) per thread per token
   static constexpr int kQ8 = 4 * kWPT;                     // int8 Q fragments (hi or lo) per thread
   static constexpr int kUPT = D / 64;                      // V units (8 dims) per thread
   static constexpr int kVW = kUPT > 1 ? kUPT / 2 : 1;      // V code words per thread per token
-  static constexpr int kTernCap = kHalf / (4 * D) < kMaxPages ? kHalf / (4 * D) : kMaxPages;
-  static constexpr int kFp8Cap = kHalf / (16 * D);
-  static constexpr int kBf16Rows = kHalf / (2 * D) >= 16 ? 16 : 8;   // token rows of a BF16 page per entry
+  static constexpr int kTernCap = kHeadHalf / (4 * D) < kMaxPages ? kHeadHalf / (4 * D) : kMaxPages;
+  static constexpr int kFp8Cap = kHeadHalf / (16 * D);
+  static constexpr int kBf16Rows = kHeadHalf / (2 * D) >= 16 ? 16 : 8;   // token rows of a BF16 page per entry
   static constexpr int kQBytes = 2 * kSteps * 32 * 4;      // per-warp f16 Q fragments
-  static_assert(kTernCap >= 1 && kFp8Cap >= 1 && kHalf >= 8 * 2 * D, "an entry must hold one page of each format");
+  static_assert(kTernCap >= 1 && kFp8Cap >= 1 && kHeadHalf >= 8 * 2 * D, "an entry must hold one page of each format");
 };
 
 __host__ __device__ constexpr int group_bytes(int fmt, int d) {
@@ -193,11 +201,11 @@ __device__ __forceinline__ T lds(const unsigned char* p) {
 }
 
 // ------------------------------------------------------- work partition
-// Sequence b contributes Hkv * np(b) units (page of one KV head), ordered
-// (b, g, j).  Each unit carries a weight: the high-precision format's cost
-// for sink and window pages, the ternary cost for older pages (anchors are
-// counted as ternary).  Warp W of NW owns the units whose weighted start
-// lies in [W*C/NW, (W+1)*C/NW), C the total weight.
+// Sequence b contributes (Hkv / HPC) * np(b) units (one page of a group of
+// HPC KV heads), ordered (b, q, j).  Each unit carries a weight: the
+// high-precision format's cost for sink and window pages, the ternary cost
+// for older pages (anchors are counted as ternary).  CTA W of NW owns the
+// units whose weighted start lies in [W*C/NW, (W+1)*C/NW), C the total weight.
 struct SeqShape {
   int np, ns, jw2, cost;   // pages, sink pages, first window page (>= ns), weight per KV head
 };
@@ -251,17 +259,17 @@ struct Prologue {
     const int b = find(seqC, c);
     const SeqShape s = seq_shape(seqL[b], sink, window, whp);
     const int cl = (int)(c - seqC[b]);
-    const int g = cl / s.cost;
-    const int j = page_of_cost(s, cl - g * s.cost, whp);
-    return seqP[b] + g * s.np + j;
+    const int q = cl / s.cost;
+    const int j = page_of_cost(s, cl - q * s.cost, whp);
+    return seqP[b] + q * s.np + j;
   }
   // worker that owns unit x
   __device__ int worker_of(int x) const {
     const int b = find(seqP, x);
     const SeqShape s = seq_shape(seqL[b], sink, window, whp);
     const int off = x - seqP[b];
-    const int g = off / s.np;
-    const long long cs = seqC[b] + (long long)g * s.cost + cost_of_page(s, off - g * s.np, whp);
+    const int q = off / s.np;
+    const long long cs = seqC[b] + (long long)q * s.cost + cost_of_page(s, off - q * s.np, whp);
     return (int)(((cs + 1) * nwg + C - 1) / C) - 1;
   }
 };
@@ -269,9 +277,11 @@ struct Prologue {
 // ------------------------------------------------------------- metadata
 // Per-lane page metadata.  Phase A (block-table slot, caller tag) is loaded
 // one chunk of 32 units ahead; phase B (format, scales) once those loads
-// have landed.  Packed words keep the register footprint small:
-//   A.info: ntok (5 bits) | is_hp (1) << 5 | g (7) << 6 | bg << 13
-//   Meta.m: fmt (2 bits) | ntok (5) << 2 | bg << 7     (m < 0: no unit)
+// have landed.  Every warp of a CTA decodes the same units (same pages and
+// formats) with the scales of its own KV head.  Packed words keep the
+// register footprint small (bq: the (sequence, head group) pair):
+//   A.info: ntok (5 bits) | is_hp (1) << 5 | g (7) << 6 | bq << 13
+//   Meta.m: fmt (2 bits) | ntok (5) << 2 | bq << 7     (m < 0: no unit)
 __device__ __forceinline__ int meta_pack(int fmt, int ntok, int bg) { return fmt | (ntok << 2) | (bg << 7); }
 __device__ __forceinline__ int meta_fmt(int m) { return m & 3; }
 __device__ __forceinline__ int meta_ntok(int m) { return (m >> 2) & 31; }
@@ -281,8 +291,8 @@ struct MetaA {
   int phys, older, info;    // info < 0: no unit
 };
 struct Meta {
-  int m;                    // packed fmt / ntok / bg
-  int grp;                  // (page slot) * Hkv + g: index of the (page, head) group
+  int m;                    // packed fmt / ntok / bq
+  int grp;                  // (page slot) * Hkv + g: index of this warp's (page, head) group
   float ks, vs;             // K / V scale of the page (gamma, s or 1)
 };
 
@@ -290,7 +300,7 @@ struct Meta {
 // x0.  The chunk's first unit is decoded once for the warp; lanes past the
 // end of that (sequence, KV head) decode their own unit.
 __device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prologue& pr, int x0, int u1,
-                                             int lane, MetaA& a) {
+                                             int lane, int hpc, int wi, MetaA& a) {
   a.info = -1;
   a.phys = 0;
   a.older = KVC_FMT_TERNARY2;
@@ -299,23 +309,25 @@ __device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prolog
   const int L0 = pr.seqL[b0];
   const int np0 = (L0 + kPage - 1) / kPage;
   const int off0 = x0 - pr.seqP[b0];
-  const int g0 = off0 / np0;
-  const int j0 = off0 - g0 * np0;
+  const int q0 = off0 / np0;
+  const int j0 = off0 - q0 * np0;
   const int x = x0 + lane;
   if (x >= u1) return;
-  int b = b0, g = g0, j = j0 + lane, L = L0;
-  if (j >= np0) {                                  // past the first (sequence, KV head)
+  int b = b0, q = q0, j = j0 + lane, L = L0;
+  if (j >= np0) {                                  // past the first (sequence, head group)
     b = pr.find(pr.seqP, x);
     L = pr.seqL[b];
     const int np = (L + kPage - 1) / kPage;
     const int off = x - pr.seqP[b];
-    g = off / np;
-    j = off - g * np;
+    q = off / np;
+    j = off - q * np;
   }
+  const int g = q * hpc + wi;                      // this warp's KV head
+  const int bq = b * (p.Hkv / hpc) + q;            // (sequence, head group) pair
   const long long row = (long long)b * p.max_pages + j;
   const int last_valid = min((j + 1) * kPage, L) - 1;
   const int is_hp = (j * kPage < p.sink || last_valid >= L - p.window) ? 1 : 0;
-  a.info = min(kPage, L - j * kPage) | (is_hp << 5) | (g << 6) | ((b * p.Hkv + g) << 13);
+  a.info = min(kPage, L - j * kPage) | (is_hp << 5) | (g << 6) | (bq << 13);
   a.phys = __ldg(p.block_table + row);
   a.older = p.older_fmt ? (int)__ldg(p.older_fmt + row) : KVC_FMT_TERNARY2;
 }
@@ -332,7 +344,8 @@ __device__ __forceinline__ void meta_phase_b(const DecodeParams& p, const MetaA&
   if (fmt < 0 || fmt > 2) {
     atomicOr(p.err, kErrFormat);
     fmt = kSkip;
-  } else if (a.phys < 0 || a.phys >= p.cache.n_pages[fmt]) {
+  } else if (a.phys < 0 || a.phys >= (fmt == KVC_FMT_BF16 ? p.cache.n_pages[0]
+                                       : fmt == KVC_FMT_FP8_E4M3 ? p.cache.n_pages[1] : p.cache.n_pages[2])) {
     atomicOr(p.err, kErrBlockTable);
     fmt = kSkip;
   } else {
@@ -360,19 +373,19 @@ struct MergeArgs {          // what the merge needs, passed by value
   int G, Hq, Hkv;
 };
 
+// Partial record k of the pair is at index rec0 + k * rstride.
 template <int D>
-__device__ __noinline__ void merge_partials(MergeArgs p, int bg, int w_first, int w_last, int lane) {
+__device__ __noinline__ void merge_partials(MergeArgs p, int bg, int rec0, int rstride, int nrec, int lane) {
   const int G = p.G;
   const int rs = G * (D + 2);
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-  const int nrec = w_last - w_first + 1;
   // row maxima and normalisers
   float ms[8], ls[8];
 #pragma unroll
   for (int r = 0; r < 8; ++r) { ms[r] = -INFINITY; ls[r] = 0.f; }
   for (int k0 = 0; k0 < nrec; k0 += 32) {
     const int k = k0 + lane;
-    const float* st = p.partials + (long long)(w_first + k + bg) * rs;
+    const float* st = p.partials + (long long)(rec0 + k * rstride) * rs;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       float mk = -INFINITY;
@@ -384,7 +397,7 @@ __device__ __noinline__ void merge_partials(MergeArgs p, int bg, int w_first, in
   }
   for (int k0 = 0; k0 < nrec; k0 += 32) {
     const int k = k0 + lane;
-    const float* st = p.partials + (long long)(w_first + k + bg) * rs;
+    const float* st = p.partials + (long long)(rec0 + k * rstride) * rs;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       float lk = 0.f;
@@ -406,12 +419,12 @@ __device__ __noinline__ void merge_partials(MergeArgs p, int bg, int w_first, in
       for (int k0 = 0; k0 < nrec; k0 += 32) {
         const int k = k0 + lane;
         float f = 0.f;
-        if (k < nrec) f = ex2(__ldcg(p.partials + (long long)(w_first + k + bg) * rs + r * (D + 2)) - ms[r]);
+        if (k < nrec) f = ex2(__ldcg(p.partials + (long long)(rec0 + k * rstride) * rs + r * (D + 2)) - ms[r]);
         const int kn = min(32, nrec - k0);
 #pragma unroll 4
         for (int kk = 0; kk < kn; ++kk) {
           const float fk = __shfl_sync(kFull, f, kk);
-          const float* row = p.partials + (long long)(w_first + k0 + kk + bg) * rs + r * (D + 2) + 2 + lane * DPL;
+          const float* row = p.partials + (long long)(rec0 + (k0 + kk) * rstride) * rs + r * (D + 2) + 2 + lane * DPL;
 #pragma unroll
           for (int i = 0; i < DPL; i += 2) {
             const float2 v = __ldcg(reinterpret_cast<const float2*>(row + i));
@@ -431,21 +444,24 @@ __device__ __noinline__ void merge_partials(MergeArgs p, int bg, int w_first, in
 
 
 // ----------------------------------------------------------- the worker
-template <int D>
+template <int D, int HPC>
 struct Worker {
-  using S = Shape<D>;
+  using S = Shape<D, HPC>;
   const DecodeParams& p;
   const Prologue& pr;
-  unsigned char* ring;     // this warp's kEntries entries
+  unsigned char* ring;     // the CTA's kEntries slots
   uint32_t* qsm;           // this warp's f16 Q fragments: [kSteps / 2][32 lanes][4]
-  Desc* desc;              // [kEntries]
-  uint64_t* bars;          // [kEntries]
+  Desc* desc;              // this warp's [kEntries] entry descriptions
+  uint64_t* bars;          // the CTA's [kEntries] slot barriers
+  int* cnt;                // the CTA's [kEntries] counts of warps done with a slot
   int lane, gid, tig;
+  int wi;                  // warp in the CTA = KV head within the group
   int u1, cursor, cb;      // unit range end, next unit to issue, chunk base
   int bf16_half;           // next half of a BF16 page to issue (half-page entries)
   Meta cur, nxt;
   MetaA nxa;
-  bool nxt_b_pending;
+  bool nxt_b_pending;       // nxt still needs phase B (its phase A loads are in nxa)
+  bool nxa_pending;         // nxa still needs phase A (the chunk after nxt)
   int W;
 
   // per (sequence, KV head) state
@@ -458,30 +474,29 @@ struct Worker {
   float m0, m1, l0, l1, uref, inv_uref;
 
   __device__ Worker(const DecodeParams& pp, const Prologue& prr, unsigned char* r, uint32_t* q, Desc* d,
-                    uint64_t* b)
-      : p(pp), pr(prr), ring(r), qsm(q), desc(d), bars(b) {}
+                    uint64_t* b, int w)
+      : p(pp), pr(prr), ring(r), qsm(q), desc(d), bars(b), wi(w) {}
+  __device__ void set_counts(int* c) { cnt = c; }
 
   __device__ __forceinline__ int shfl(int v, int src) { return __shfl_sync(kFull, v, src); }
   __device__ __forceinline__ float shflf(float v, int src) { return __shfl_sync(kFull, v, src); }
 
-  // Fill ring slot `slot` with the next entry; false when the warp's units
-  // are exhausted.
-  __device__ bool issue(int slot) {
+  // Describe the next entry of the CTA's unit range in this warp's desc[slot]
+  // (every warp of the CTA forms the same entries); with `copy`, also fill
+  // ring slot `slot` for all HPC heads.  False when the range is exhausted.
+  __device__ bool issue(int slot, bool copy) {
     if (cursor >= u1) return false;
     int li = cursor - cb;
     if (li >= 32) {
-      if (nxt_b_pending) meta_phase_b(p, nxa, nxt);
+      if (nxt_b_pending) meta_phase_b(p, nxa, nxt);   // only when a chunk took one entry
       cur = nxt;
       cb += 32;
       li -= 32;
-      meta_phase_a(p, pr, cb + 32, u1, lane, nxa);
-      nxt_b_pending = true;
-    } else if (nxt_b_pending) {
-      meta_phase_b(p, nxa, nxt);
       nxt_b_pending = false;
+      nxa_pending = true;
     }
     const int m0l = shfl(cur.m, li);
-    const int f0 = meta_fmt(m0l), bg0 = meta_bg(m0l);
+    const int f0 = meta_fmt(m0l), bg0 = meta_bg(m0l) * HPC + wi;   // this warp's (sequence, KV head)
     int np = 1, row0 = 0, nrows, advance = 1;
     int bytes_per_page = 0, src_off = 0;
     if (f0 == KVC_FMT_BF16 && S::kBf16Rows == 8) {
@@ -526,28 +541,51 @@ struct Worker {
       d.vs[k] = cur.vs;
     }
     __syncwarp();
-    fence_proxy_async();
-    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], f0 == kSkip ? 0u : (uint32_t)(2 * np * bytes_per_page));
-    __syncwarp();
-    if (f0 != kSkip && mine) {
-      const unsigned char* kb;
-      const unsigned char* vb;
-      if (f0 == KVC_FMT_TERNARY2) {
-        kb = static_cast<const unsigned char*>(p.cache.k_tern);
-        vb = static_cast<const unsigned char*>(p.cache.v_tern);
-      } else if (f0 == KVC_FMT_FP8_E4M3) {
-        kb = static_cast<const unsigned char*>(p.cache.k_fp8);
-        vb = static_cast<const unsigned char*>(p.cache.v_fp8);
-      } else {
-        kb = static_cast<const unsigned char*>(p.cache.k_bf16);
-        vb = static_cast<const unsigned char*>(p.cache.v_bf16);
+    if (copy) {
+      // the HPC heads' groups of a page are contiguous: one copy per page
+      // for K and one for V (BF16 half pages: one per head, 8 rows each)
+      const bool half = f0 == KVC_FMT_BF16 && S::kBf16Rows == 8;
+      const int per = half ? 8 * 2 * D : HPC * bytes_per_page;   // bytes per copy
+      const int ncopy = f0 == kSkip ? 0 : (half ? HPC : np);
+      fence_proxy_async();
+      if (lane == 0) mbar_arrive_expect_tx(&bars[slot], (uint32_t)(2 * ncopy * per));
+      __syncwarp();
+      const int src_lane = half ? li : li + lane;
+      const int grp = shfl(cur.grp, min(src_lane, 31)) - wi;       // group of head 0 of the CTA
+      if (lane < ncopy) {
+        const unsigned char* kb;
+        const unsigned char* vb;
+        if (f0 == KVC_FMT_TERNARY2) {
+          kb = static_cast<const unsigned char*>(p.cache.k_tern);
+          vb = static_cast<const unsigned char*>(p.cache.v_tern);
+        } else if (f0 == KVC_FMT_FP8_E4M3) {
+          kb = static_cast<const unsigned char*>(p.cache.k_fp8);
+          vb = static_cast<const unsigned char*>(p.cache.v_fp8);
+        } else {
+          kb = static_cast<const unsigned char*>(p.cache.k_bf16);
+          vb = static_cast<const unsigned char*>(p.cache.v_bf16);
+        }
+        const int gb = group_bytes(f0, D);
+        const long long off = half ? (long long)(grp + lane) * gb + src_off : (long long)grp * gb;
+        unsigned char* e = ring + slot * S::kSlotBytes + lane * per;
+        bulk_g2s(e, kb + off, (uint32_t)per, &bars[slot]);
+        bulk_g2s(e + S::kHalf, vb + off, (uint32_t)per, &bars[slot]);
       }
-      const long long off = (long long)cur.grp * group_bytes(f0, D) + src_off;
-      unsigned char* e = ring + slot * S::kEntryBytes + k * bytes_per_page;
-      bulk_g2s(e, kb + off, (uint32_t)bytes_per_page, &bars[slot]);
-      bulk_g2s(e + S::kHalf, vb + off, (uint32_t)bytes_per_page, &bars[slot]);
     }
     cursor += advance;
+    // Metadata prefetch for the next chunk, issued only after this entry's
+    // copies: the proxy fence above would otherwise wait for these global
+    // loads.  Phase B (which reads phase A's block-table entries) waits until
+    // three quarters of the current chunk are issued, so those loads have
+    // landed; its scale loads are first used at the next chunk switch.
+    if (nxa_pending) {
+      meta_phase_a(p, pr, cb + 32, u1, lane, HPC, wi, nxa);
+      nxa_pending = false;
+      nxt_b_pending = true;
+    } else if (nxt_b_pending && cursor - cb >= 24) {
+      meta_phase_b(p, nxa, nxt);
+      nxt_b_pending = false;
+    }
     return true;
   }
 
@@ -630,7 +668,10 @@ struct Worker {
       l1 += __shfl_xor_sync(kFull, l1, o);
     }
     const int rs = G * (D + 2);
-    float* rec = p.partials + (long long)(W + bg) * rs;
+    // record of (CTA W, pair bq, head wi): records of consecutive CTAs of a
+    // pair are HPC apart, and distinct pairs never collide
+    const int bq = bg / HPC;
+    float* rec = p.partials + (long long)((W + bq) * HPC + wi) * rs;
     const int c0 = 2 * tig, c1 = 2 * tig + 1;
     if (gid == 0) {
       if (c0 < G) { rec[c0 * (D + 2)] = m0; rec[c0 * (D + 2) + 1] = l0; }
@@ -652,16 +693,17 @@ struct Worker {
     }
     __threadfence();
     __syncwarp();
-    const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+    const int b = bg / p.Hkv, q = (bg - b * p.Hkv) / HPC;
     const int np = (pr.seqL[b] + kPage - 1) / kPage;
-    const int x0 = pr.seqP[b] + g * np;
+    const int x0 = pr.seqP[b] + q * np;
     const int w_first = pr.worker_of(x0), w_last = pr.worker_of(x0 + np - 1);
     unsigned last = 0;
     if (lane == 0) last = atomicAdd(p.tickets + bg, 1u) == (unsigned)(w_last - w_first);
     last = __shfl_sync(kFull, last, 0);
     if (!last) return;
     __threadfence();
-    merge_partials<D>(MergeArgs{p.partials, p.out, p.tickets, p.G, p.Hq, p.Hkv}, bg, w_first, w_last, lane);
+    merge_partials<D>(MergeArgs{p.partials, p.out, p.tickets, p.G, p.Hq, p.Hkv}, bg, (w_first + bq) * HPC + wi,
+                      HPC, w_last - w_first + 1, lane);
   }
 
   // ---------------------------------------------------------- Q . K^T
@@ -861,8 +903,7 @@ struct Worker {
   template <bool SPLIT>
   // sc0 / sc1 scale the thread's two score columns (s[0], s[2] and s[1], s[3]).
   __device__ __forceinline__ void softmax_page(float (&s)[4], float sc0, float sc1, float ratio, int nt,
-                                               float c0f, float c1f, uint32_t& b0, uint32_t& b1, uint32_t& lo0,
-                                               uint32_t& lo1) {
+                                               uint32_t& b0, uint32_t& b1, uint32_t& lo0, uint32_t& lo1) {
     // exponent arguments s*sc - m; the scales are >= 0 (gamma, s or 1, times max|q|)
     float mx0 = fmaxf(s[0], s[2]) * sc0, mx1 = fmaxf(s[1], s[3]) * sc1;
     bool masked = false;
@@ -902,10 +943,8 @@ struct Worker {
     const float p00 = ex2(e00), p01 = ex2(e01), p10 = ex2(e10), p11 = ex2(e11);
     l0 += p00 + p10;
     l1 += p01 + p11;
-    // P scaled by the page's V scale (relative to the reference); padded GQA
-    // columns (>= G) get P = 0
-    const float q0 = c0f * ratio, q1 = c1f * ratio;
-    const float y00 = p00 * q0, y01 = p01 * q1, y10 = p10 * q0, y11 = p11 * q1;
+    // P scaled by the page's V scale (relative to the reference)
+    const float y00 = p00 * ratio, y01 = p01 * ratio, y10 = p10 * ratio, y11 = p11 * ratio;
     const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
     b0 = movtrans(h0);
     b1 = movtrans(h1);
@@ -939,12 +978,16 @@ struct Worker {
   }
 
   // --------------------------------------------------------- one entry
+  // e: the ring slot.  Page i of this warp's head starts at
+  // e + (i * HPC + wi) * GB (K) and kHalf further (V).  Columns of padded
+  // GQA rows (query heads >= G, Q = 0) run along with finite values and are
+  // never written out.
   __device__ __forceinline__ void process(const unsigned char* e, const Desc& d) {
     const int fmt = d.fmt, np = d.np;
-    const float c0f = 2 * tig < p.G ? 1.f : 0.f, c1f = 2 * tig + 1 < p.G ? 1.f : 0.f;
     uint32_t b0, b1, lo0 = 0u, lo1 = 0u;
     if (fmt == KVC_FMT_TERNARY2) {
-      constexpr int GB = group_bytes(KVC_FMT_TERNARY2, D);
+      constexpr int GB = HPC * group_bytes(KVC_FMT_TERNARY2, D);   // page stride
+      e += wi * group_bytes(KVC_FMT_TERNARY2, D);
       rebase_value_scale(d, 0.5f);
       const float vf = 0.5f * inv_uref;
       // software pipeline: the scores of page i+1 are computed while page i
@@ -956,34 +999,36 @@ struct Worker {
       for (; i + 1 < np; ++i) {
         float sn[4];
         qk_ternary(e + (i + 1) * GB, sn);
-        softmax_page<false>(s, d.ks[i] * kq0, d.ks[i] * kq1, d.vs[i] * vf, kPage, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<false>(s, d.ks[i] * kq0, d.ks[i] * kq1, d.vs[i] * vf, kPage, b0, b1, lo0, lo1);
         pv_ternary(e + S::kHalf + i * GB, b0, b1, kPage);
 #pragma unroll
         for (int c = 0; c < 4; ++c) s[c] = sn[c];
       }
-      softmax_page<false>(s, d.ks[i] * kq0, d.ks[i] * kq1, d.vs[i] * vf, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+      softmax_page<false>(s, d.ks[i] * kq0, d.ks[i] * kq1, d.vs[i] * vf, d.nrows, b0, b1, lo0, lo1);
       pv_ternary(e + S::kHalf + i * GB, b0, b1, d.nrows);
     } else if (fmt == KVC_FMT_FP8_E4M3) {
-      constexpr int GB = group_bytes(KVC_FMT_FP8_E4M3, D);
+      constexpr int GB = HPC * group_bytes(KVC_FMT_FP8_E4M3, D);
+      e += wi * group_bytes(KVC_FMT_FP8_E4M3, D);
       rebase_value_scale(d, 1.f);
       for (int i = 0; i < np; ++i) {
         const int nt = i == np - 1 ? d.nrows : kPage;
         float s[4];
         qk_fp8(e + i * GB, s);
         const float sc = d.ks[i] * p.scale_log2;
-        softmax_page<true>(s, sc, sc, d.vs[i] * inv_uref, nt, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<true>(s, sc, sc, d.vs[i] * inv_uref, nt, b0, b1, lo0, lo1);
         pv_fp8(e + S::kHalf + i * GB, b0, b1, lo0, lo1, nt);
       }
     } else if (fmt == KVC_FMT_BF16) {
       rebase_value_scale(d, 1.f);
+      e += wi * S::kBf16Rows * 2 * D;        // full page, or the 8 rows of a half page
       float s[4];
       if constexpr (S::kBf16Rows == 16) {
         qk_bf16<16>(e, s);
-        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, b0, b1, lo0, lo1);
         pv_bf16<16>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       } else {
         qk_bf16<8>(e, s);
-        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, c0f, c1f, b0, b1, lo0, lo1);
+        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, b0, b1, lo0, lo1);
         pv_bf16<8>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       }
     }
@@ -998,9 +1043,27 @@ struct Worker {
       finish();
       begin(bg);
     }
-    if (d.fmt != kSkip) process(ring + slot * S::kEntryBytes, d);
+    if (d.fmt != kSkip) process(ring + slot * S::kSlotBytes, d);
     __syncwarp();
     return true;
+  }
+
+  // This warp is done reading ring slot `slot`.  True for the last of the
+  // CTA's warps to get here, which then refills the slot (no warp waits for
+  // another: the refill happens after every warp's reads of the slot).
+  __device__ __forceinline__ bool release(int slot) {
+    if constexpr (HPC == 1) {
+      return true;
+    } else {
+      unsigned last = 0;
+      // the warp's reads of the slot have completed (their values are in
+      // registers and __syncwarp ordered them before this point)
+      if (lane == 0) {
+        last = atomicAdd(&cnt[slot], 1) == HPC - 1;
+        if (last) cnt[slot] = 0;
+      }
+      return __shfl_sync(kFull, last, 0) != 0u;
+    }
   }
 
   __device__ void run(int w_index) {
@@ -1016,19 +1079,21 @@ struct Worker {
     cur_bg = -1;
     {
       MetaA a;
-      meta_phase_a(p, pr, cb, u1, lane, a);
+      meta_phase_a(p, pr, cb, u1, lane, HPC, wi, a);
       meta_phase_b(p, a, cur);
     }
-    meta_phase_a(p, pr, cb + 32, u1, lane, nxa);
+    meta_phase_a(p, pr, cb + 32, u1, lane, HPC, wi, nxa);
     nxt_b_pending = true;
+    nxa_pending = false;
 
-    bool v0 = issue(0), v1 = issue(1);
+    // warp 0 fills both slots first; later refills come from release()
+    bool v0 = issue(0, wi == 0), v1 = issue(1, wi == 0);
     bool ok = true;
     for (int it = 0;; ++it) {          // one call site: the hot loop stays compact
       const int slot = it & 1;
       if (!(slot ? v1 : v0)) break;
       if (!(ok = consume(slot, (uint32_t)(it >> 1) & 1u))) break;
-      const bool nv = issue(slot);
+      const bool nv = issue(slot, release(slot));
       if (slot) v1 = nv; else v0 = nv;
     }
     if (!ok) {
@@ -1042,21 +1107,26 @@ struct Worker {
   }
 };
 
-template <int D>
-__global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) {
-  using S = Shape<D>;
+template <int D, int HPC>
+__global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
+  using S = Shape<D, HPC>;
   extern __shared__ __align__(128) unsigned char smem[];
   unsigned char* ring = smem;
-  uint32_t* qbuf = reinterpret_cast<uint32_t*>(smem + kWarps * kEntries * S::kEntryBytes);
-  Desc* descs = reinterpret_cast<Desc*>(smem + kWarps * kEntries * S::kEntryBytes + kWarps * S::kQBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(descs + kWarps * kEntries);
-  int* seqP = reinterpret_cast<int*>(bars + kWarps * kEntries);
+  uint32_t* qbuf = reinterpret_cast<uint32_t*>(smem + kEntries * S::kSlotBytes);
+  Desc* descs = reinterpret_cast<Desc*>(smem + kEntries * S::kSlotBytes + HPC * S::kQBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(descs + HPC * kEntries);
+  int* cnt = reinterpret_cast<int*>(bars + kEntries);
+  int* seqP = cnt + kEntries;
   int* seqC = seqP + (p.B + 1);
   int* seqL = seqC + (p.B + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int whp = p.hp == KVC_FMT_BF16 ? kCostBf16 : kCostFp8;
+  const int whp = p.hp == KVC_FMT_BF16 ? cost_bf16<D>() : kCostFp8;
+  const int nq = p.Hkv / HPC;          // head groups per sequence
 
-  if (threadIdx.x < kWarps * kEntries) mbar_init(&bars[threadIdx.x], 1);
+  if (threadIdx.x < kEntries) {
+    mbar_init(&bars[threadIdx.x], 1);
+    cnt[threadIdx.x] = 0;
+  }
   if (warp == 0) {
     int carry_u = 0, carry_c = 0;
     for (int base = 0; base < p.B; base += 32) {
@@ -1070,8 +1140,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
         }
         seqL[b] = L;
         const SeqShape s = seq_shape(L, p.sink, p.window, whp);
-        u = s.np * p.Hkv;
-        c = s.cost * p.Hkv;
+        u = s.np * nq;
+        c = s.cost * nq;
       }
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -1109,26 +1179,27 @@ __global__ void __launch_bounds__(kWarps * 32) decode_tc_kernel(DecodeParams p) 
   // every worker's weight range is at least twice the heaviest unit, so
   // each one owns at least one unit
   const long long most = pr.C / (2 * kCostBf16);
-  pr.nwg = (int)((long long)p.n_splits < most ? p.n_splits : (most > 0 ? most : 1));
-  const int W = blockIdx.x * kWarps + warp;
+  pr.nwg = (int)((long long)gridDim.x < most ? gridDim.x : (most > 0 ? most : 1));
+  const int W = blockIdx.x;
   if (W >= pr.nwg) return;
-  Worker<D> wk(p, pr, ring + warp * kEntries * S::kEntryBytes, qbuf + warp * (S::kQBytes / 4),
-               descs + warp * kEntries, bars + warp * kEntries);
+  Worker<D, HPC> wk(p, pr, ring, qbuf + warp * (S::kQBytes / 4), descs + warp * kEntries, bars, warp);
+  wk.set_counts(cnt);
   wk.run(W);
 }
 
-template <int D>
+template <int D, int HPC>
 size_t tc_smem_bytes(int batch) {
-  return (size_t)kWarps * kEntries * Shape<D>::kEntryBytes + (size_t)kWarps * Shape<D>::kQBytes +
-         kWarps * kEntries * sizeof(Desc) +
-         kWarps * kEntries * sizeof(uint64_t) + (size_t)(3 * batch + 2) * sizeof(int);
+  using S = Shape<D, HPC>;
+  return (size_t)kEntries * S::kSlotBytes + (size_t)HPC * S::kQBytes + HPC * kEntries * sizeof(Desc) +
+         kEntries * sizeof(uint64_t) + kEntries * sizeof(int) + (size_t)(3 * batch + 2) * sizeof(int);
 }
 
 // The kernel's shared memory depends on the batch (the sequence tables); the
 // largest size is opted into once per device, and CTAs per SM are cached per
-// (device, head_dim, batch) so a call costs no runtime query after the first.
+// (device, head_dim, heads per CTA, batch) so a call costs no runtime query
+// after the first.
 constexpr int kMaxDev = 64;
-template <int D>
+template <int D, int HPC>
 cudaError_t tc_occupancy(int batch, int* ctas_per_sm) {
   static std::mutex mu;
   static bool opted[kMaxDev] = {};
@@ -1144,15 +1215,34 @@ cudaError_t tc_occupancy(int batch, int* ctas_per_sm) {
     return cudaSuccess;
   }
   if (dev >= 0 && dev < kMaxDev && !opted[dev]) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tc_smem_bytes<D>(kTcMaxBatchTpl));
+    e = cudaFuncSetAttribute(decode_tc_kernel<D, HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc_smem_bytes<D, HPC>(kTcMaxBatchTpl));
     if (e != cudaSuccess) return e;
     opted[dev] = true;
   }
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D>, kWarps * 32,
-                                                    tc_smem_bytes<D>(batch));
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D, HPC>, HPC * 32,
+                                                    tc_smem_bytes<D, HPC>(batch));
   if (e == cudaSuccess) cache[key] = *ctas_per_sm;
   return e;
+}
+
+template <int D>
+cudaError_t tc_occupancy_hpc(int hpc, int batch, int* ctas_per_sm) {
+  switch (hpc) {
+    case 1: return tc_occupancy<D, 1>(batch, ctas_per_sm);
+    case 2: return tc_occupancy<D, 2>(batch, ctas_per_sm);
+    case 4: return tc_occupancy<D, 4>(batch, ctas_per_sm);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D>
+void launch_tc(const DecodeParams& p, int hpc, int grid, cudaStream_t s) {
+  switch (hpc) {
+    case 1: decode_tc_kernel<D, 1><<<grid, 32, tc_smem_bytes<D, 1>(p.B), s>>>(p); break;
+    case 2: decode_tc_kernel<D, 2><<<grid, 64, tc_smem_bytes<D, 2>(p.B), s>>>(p); break;
+    default: decode_tc_kernel<D, 4><<<grid, 128, tc_smem_bytes<D, 4>(p.B), s>>>(p); break;
+  }
 }
 
 }  // namespace
@@ -1165,16 +1255,20 @@ bool tc_supported(int batch, int hkv, int max_pages) {
   return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages * kCostBf16 < (1ll << 31);
 }
 
-cudaError_t tc_grid(int batch, int d, int* grid) {
+// KV heads per CTA: the largest of 4, 2, 1 that divides Hkv.
+int tc_heads_per_cta(int hkv) { return hkv % 4 == 0 ? 4 : (hkv % 2 == 0 ? 2 : 1); }
+
+cudaError_t tc_grid(int batch, int d, int hkv, int* grid) {
   int dev = 0, sms = 0, per = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  const int hpc = tc_heads_per_cta(hkv);
   switch (d) {
-    case 64: e = tc_occupancy<64>(batch, &per); break;
-    case 128: e = tc_occupancy<128>(batch, &per); break;
-    case 256: e = tc_occupancy<256>(batch, &per); break;
+    case 64: e = tc_occupancy_hpc<64>(hpc, batch, &per); break;
+    case 128: e = tc_occupancy_hpc<128>(hpc, batch, &per); break;
+    case 256: e = tc_occupancy_hpc<256>(hpc, batch, &per); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
@@ -1182,13 +1276,14 @@ cudaError_t tc_grid(int batch, int d, int* grid) {
   return cudaSuccess;
 }
 
-int tc_warps_per_cta() { return kWarps; }
+int tc_warps_per_cta(int hkv) { return tc_heads_per_cta(hkv); }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s) {
+  const int hpc = tc_heads_per_cta(p.Hkv);
   switch (head_dim) {
-    case 64: decode_tc_kernel<64><<<grid, kWarps * 32, tc_smem_bytes<64>(p.B), s>>>(p); break;
-    case 128: decode_tc_kernel<128><<<grid, kWarps * 32, tc_smem_bytes<128>(p.B), s>>>(p); break;
-    case 256: decode_tc_kernel<256><<<grid, kWarps * 32, tc_smem_bytes<256>(p.B), s>>>(p); break;
+    case 64: launch_tc<64>(p, hpc, grid, s); break;
+    case 128: launch_tc<128>(p, hpc, grid, s); break;
+    case 256: launch_tc<256>(p, hpc, grid, s); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

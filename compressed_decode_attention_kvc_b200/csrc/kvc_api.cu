@@ -45,11 +45,11 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
     // persistent grid, every warp a stream-K worker; one partial state per
     // (warp, pair) boundary: at most warps + pairs records
     int grid = 0;
-    cudaError_t e = tc_grid(batch, d, &grid);
+    cudaError_t e = tc_grid(batch, d, hkv, &grid);
     if (e != cudaSuccess) return e;
     plan->tensor_cores = true;
     plan->grid = grid;
-    plan->n_splits = grid * tc_warps_per_cta();
+    plan->n_splits = grid * tc_warps_per_cta(hkv);
     plan->pages_per_split = 0;
     plan->bytes = plan->partial_offset + ((size_t)plan->n_splits + (size_t)bg) * record;
     return cudaSuccess;
