@@ -180,6 +180,11 @@ __device__ __forceinline__ uint32_t tern2(uint32_t w, int o) {
 __device__ __forceinline__ uint32_t tern8(uint32_t w, int f) {
   return (f == 3 ? w : (w << (6 - 2 * f))) & 0xC0C0C0C0u;
 }
+// y as an f16 pair (hi, lo) with hi = f16(y), lo = f16(y - hi): ~22 bits.
+__device__ __forceinline__ uint32_t split_f16x2(float y) {
+  const float hi = __half2float(__float2half_rn(y));
+  return f16x2(hi, y - hi);
+}
 // Two e4m3 bytes (low byte -> low half) -> f16x2.
 __device__ __forceinline__ uint32_t e4m3x2_f16(uint32_t two_bytes) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xFFFFu), __NV_E4M3);
@@ -444,7 +449,12 @@ __device__ __noinline__ void merge_partials(MergeArgs p, int bg, int rec0, int r
 
 
 // ----------------------------------------------------------- the worker
-template <int D, int HPC>
+// NARROW (GQA group of at most 4 query heads): MMA column 2h + part belongs
+// to query head h.  In Q.K^T of ternary pages the two parts are Q's int8 hi
+// and lo (one int8 MMA per k-step instead of two); in P.V they are P's f16
+// hi and lo (one MMA per m-tile carries the split P); elsewhere part 1 is 0.
+// Otherwise (WIDE, up to 8 query heads) column n is query head n.
+template <int D, int HPC, bool NARROW>
 struct Worker {
   using S = Shape<D, HPC>;
   const DecodeParams& p;
@@ -468,8 +478,9 @@ struct Worker {
   int cur_bg;
   // Q of the group as int8 hi/lo fragments for ternary pages:
   // q ~= sq * (128 * hi + lo), sq = max|q| / 16256 per query head
-  uint32_t qh[S::kQ8], ql[S::kQ8];
-  float kq0, kq1;          // score scale of the thread's two columns: sq * log2(e) * softmax_scale / 64
+  // (NARROW: qh holds this thread's column, hi or lo of one head)
+  uint32_t qh[S::kQ8], ql[NARROW ? 1 : S::kQ8];
+  float kq0, kq1;          // score scale of the thread's score columns: sq * log2(e) * softmax_scale / 64
   float acc[S::kSteps][4];
   float m0, m1, l0, l1, uref, inv_uref;
 
@@ -593,7 +604,7 @@ struct Worker {
   __device__ void begin(int bg) {
     cur_bg = bg;
     const int b = bg / p.Hkv, g = bg - (bg / p.Hkv) * p.Hkv;
-    const int r = gid;                       // query head within the group
+    const int r = NARROW ? gid >> 1 : gid;   // query head within the group
     uint32_t raw[S::kWPT * 8];               // 16 * kWPT bf16 of row r
     if (r < p.G) {
       const uint4* src = reinterpret_cast<const uint4*>(
@@ -614,7 +625,8 @@ struct Worker {
     for (int ri = 0; ri < 2 * S::kSteps; ++ri) {
       const int wl = ri >> 3, j = ri & 7;
       const uint32_t wa = raw[8 * wl + (j >> 1)], wb = raw[8 * wl + 4 + (j >> 1)];
-      qsm[((ri >> 2) * 32 + lane) * 4 + (ri & 3)] = bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
+      const uint32_t v = (NARROW && (gid & 1)) ? 0u : bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
+      qsm[((ri >> 2) * 32 + lane) * 4 + (ri & 3)] = v;
     }
     // int8 hi/lo B fragments for ternary pages.  Fragment j carries, in
     // byte i, the thread-local dim 16 * (j >> 2) + 4 * i + (j & 3): the dims
@@ -640,13 +652,22 @@ struct Worker {
         h |= (uint32_t)(hi & 0xFF) << (8 * i);
         l |= (uint32_t)(lo & 0xFF) << (8 * i);
       }
-      qh[j] = h;
-      ql[j] = l;
+      if constexpr (NARROW) {
+        qh[j] = (gid & 1) ? l : h;
+      } else {
+        qh[j] = h;
+        ql[j] = l;
+      }
     }
     const float sq = amax * (1.f / 16256.f);
     const float f = p.scale_log2 * (1.f / 64.f);
-    kq0 = __shfl_sync(kFull, sq, 8 * tig) * f;          // head 2 * tig (lane group gid = 2 * tig)
-    kq1 = __shfl_sync(kFull, sq, 8 * tig + 4) * f;      // head 2 * tig + 1
+    if constexpr (NARROW) {
+      kq0 = __shfl_sync(kFull, sq, 8 * tig) * f;        // head tig (lane group gid = 2 * tig)
+      kq1 = 0.f;
+    } else {
+      kq0 = __shfl_sync(kFull, sq, 8 * tig) * f;        // head 2 * tig (lane group gid = 2 * tig)
+      kq1 = __shfl_sync(kFull, sq, 8 * tig + 4) * f;    // head 2 * tig + 1
+    }
 #pragma unroll
     for (int mt = 0; mt < S::kSteps; ++mt)
 #pragma unroll
@@ -672,13 +693,28 @@ struct Worker {
     // pair are HPC apart, and distinct pairs never collide
     const int bq = bg / HPC;
     float* rec = p.partials + (long long)((W + bq) * HPC + wi) * rs;
+    if constexpr (NARROW) {
+      // head tig: columns 2 * tig (P hi) and 2 * tig + 1 (P lo) add up
+      if (tig < G) {
+        float* r = rec + tig * (D + 2);
+        if (gid == 0) { r[0] = m0; r[1] = l0; }
+#pragma unroll
+        for (int mt = 0; mt < S::kSteps; ++mt) {
+          const int la = mt, lb = mt + S::kSteps;
+          const int da = 8 * (gid * S::kUPT + (la >> 3)) + (la & 7);
+          const int db = 8 * (gid * S::kUPT + (lb >> 3)) + (lb & 7);
+          r[2 + da] = (acc[mt][0] + acc[mt][1]) * uref;
+          r[2 + db] = (acc[mt][2] + acc[mt][3]) * uref;
+        }
+      }
+    }
     const int c0 = 2 * tig, c1 = 2 * tig + 1;
-    if (gid == 0) {
+    if (!NARROW && gid == 0) {
       if (c0 < G) { rec[c0 * (D + 2)] = m0; rec[c0 * (D + 2) + 1] = l0; }
       if (c1 < G) { rec[c1 * (D + 2)] = m1; rec[c1 * (D + 2) + 1] = l1; }
     }
 #pragma unroll
-    for (int mt = 0; mt < S::kSteps; ++mt) {
+    for (int mt = 0; mt < S::kSteps && !NARROW; ++mt) {
       const int la = mt, lb = mt + S::kSteps;
       const int da = 8 * (gid * S::kUPT + (la >> 3)) + (la & 7);
       const int db = 8 * (gid * S::kUPT + (lb >> 3)) + (lb & 7);
@@ -730,11 +766,22 @@ struct Worker {
       const int j0 = 2 * st, j1 = 2 * st + 1;
       const uint32_t a0 = tern8(wa[j0 >> 2], j0 & 3), a1 = tern8(wb[j0 >> 2], j0 & 3);
       const uint32_t a2 = tern8(wa[j1 >> 2], j1 & 3), a3 = tern8(wb[j1 >> 2], j1 & 3);
-      imma16832(th, a0, a1, a2, a3, qh[j0], qh[j1]);
-      imma16832(tl, a0, a1, a2, a3, ql[j0], ql[j1]);
+      if constexpr (NARROW) {
+        imma16832((st & 1) ? tl : th, a0, a1, a2, a3, qh[j0], qh[j1]);   // two chains
+      } else {
+        imma16832(th, a0, a1, a2, a3, qh[j0], qh[j1]);
+        imma16832(tl, a0, a1, a2, a3, ql[j0], ql[j1]);
+      }
     }
+    if constexpr (NARROW) {
+      // columns (hi, lo) of head tig: s[0] token gid, s[2] token gid + 8
+      s[0] = (float)((th[0] + tl[0]) * 128 + (th[1] + tl[1]));
+      s[2] = (float)((th[2] + tl[2]) * 128 + (th[3] + tl[3]));
+      s[1] = s[3] = 0.f;
+    } else {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) s[c] = (float)(th[c] * 128 + tl[c]);
+      for (int c = 0; c < 4; ++c) s[c] = (float)(th[c] * 128 + tl[c]);
+    }
   }
 
   // f16 Q fragments of k-steps 2k and 2k + 1
@@ -864,7 +911,7 @@ struct Worker {
       const uint32_t a2 = e4m3x2_f16(prmt(x2[ia], x3[ia], sa)) & m23;
       const uint32_t a3 = e4m3x2_f16(prmt(x2[ib], x3[ib], sb)) & m23;
       mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
-      mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
+      if constexpr (!NARROW) mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
     }
   }
 
@@ -889,7 +936,7 @@ struct Worker {
         a3 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb)) & m23;
       }
       mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
-      mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
+      if constexpr (!NARROW) mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
     }
   }
 
@@ -900,10 +947,45 @@ struct Worker {
   // With SPLIT, P is passed as an f16 hi + lo pair (b0/b1 and lo0/lo1,
   // ~22 bits): pages whose values can be large (FP8, BF16) need it to keep
   // the absolute error of P.V small; ternary values are bounded by gamma.
+  // NARROW: one query head (tig) per thread, scores s[0] (token gid) and
+  // s[2] (token gid + 8) scaled by sc0; P always goes out as the hi + lo pair
+  // in columns (2 * tig, 2 * tig + 1), so SPLIT does not apply.
   template <bool SPLIT>
   // sc0 / sc1 scale the thread's two score columns (s[0], s[2] and s[1], s[3]).
   __device__ __forceinline__ void softmax_page(float (&s)[4], float sc0, float sc1, float ratio, int nt,
                                                uint32_t& b0, uint32_t& b1, uint32_t& lo0, uint32_t& lo1) {
+    if constexpr (NARROW) {
+      float mx = fmaxf(s[0], s[2]) * sc0;
+      bool masked = false;
+      if (nt < kPage) {
+        masked = true;
+        mx = gid + 8 < nt ? mx : s[0] * sc0;
+        if (gid >= nt) mx = -INFINITY;
+      }
+      if (__any_sync(kFull, mx > m0 + kTau)) {
+        float r = mx;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) r = fmaxf(r, __shfl_xor_sync(kFull, r, o));
+        const float n0 = fmaxf(m0, r);
+        const float a0 = n0 == -INFINITY ? 1.f : ex2(m0 - n0);
+#pragma unroll
+        for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[mt][c] *= a0;
+        l0 *= a0;
+        m0 = n0;
+      }
+      float e0 = fmaf(s[0], sc0, -m0), e1 = fmaf(s[2], sc0, -m0);
+      if (masked) {
+        if (gid >= nt) e0 = -INFINITY;
+        if (gid + 8 >= nt) e1 = -INFINITY;
+      }
+      const float p0 = ex2(e0), p1 = ex2(e1);
+      l0 += p0 + p1;
+      b0 = movtrans(split_f16x2(p0 * ratio));
+      b1 = movtrans(split_f16x2(p1 * ratio));
+      return;
+    }
     // exponent arguments s*sc - m; the scales are >= 0 (gamma, s or 1, times max|q|)
     float mx0 = fmaxf(s[0], s[2]) * sc0, mx1 = fmaxf(s[1], s[3]) * sc1;
     bool masked = false;
@@ -1107,7 +1189,7 @@ struct Worker {
   }
 };
 
-template <int D, int HPC>
+template <int D, int HPC, bool NARROW>
 __global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
   using S = Shape<D, HPC>;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -1182,7 +1264,7 @@ __global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
   pr.nwg = (int)((long long)gridDim.x < most ? gridDim.x : (most > 0 ? most : 1));
   const int W = blockIdx.x;
   if (W >= pr.nwg) return;
-  Worker<D, HPC> wk(p, pr, ring, qbuf + warp * (S::kQBytes / 4), descs + warp * kEntries, bars, warp);
+  Worker<D, HPC, NARROW> wk(p, pr, ring, qbuf + warp * (S::kQBytes / 4), descs + warp * kEntries, bars, warp);
   wk.set_counts(cnt);
   wk.run(W);
 }
@@ -1199,7 +1281,7 @@ size_t tc_smem_bytes(int batch) {
 // (device, head_dim, heads per CTA, batch) so a call costs no runtime query
 // after the first.
 constexpr int kMaxDev = 64;
-template <int D, int HPC>
+template <int D, int HPC, bool NARROW>
 cudaError_t tc_occupancy(int batch, int* ctas_per_sm) {
   static std::mutex mu;
   static bool opted[kMaxDev] = {};
@@ -1215,33 +1297,33 @@ cudaError_t tc_occupancy(int batch, int* ctas_per_sm) {
     return cudaSuccess;
   }
   if (dev >= 0 && dev < kMaxDev && !opted[dev]) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<D, HPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_tc_kernel<D, HPC, NARROW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)tc_smem_bytes<D, HPC>(kTcMaxBatchTpl));
     if (e != cudaSuccess) return e;
     opted[dev] = true;
   }
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D, HPC>, HPC * 32,
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, decode_tc_kernel<D, HPC, NARROW>, HPC * 32,
                                                     tc_smem_bytes<D, HPC>(batch));
   if (e == cudaSuccess) cache[key] = *ctas_per_sm;
   return e;
 }
 
-template <int D>
+template <int D, bool NARROW>
 cudaError_t tc_occupancy_hpc(int hpc, int batch, int* ctas_per_sm) {
   switch (hpc) {
-    case 1: return tc_occupancy<D, 1>(batch, ctas_per_sm);
-    case 2: return tc_occupancy<D, 2>(batch, ctas_per_sm);
-    case 4: return tc_occupancy<D, 4>(batch, ctas_per_sm);
+    case 1: return tc_occupancy<D, 1, NARROW>(batch, ctas_per_sm);
+    case 2: return tc_occupancy<D, 2, NARROW>(batch, ctas_per_sm);
+    case 4: return tc_occupancy<D, 4, NARROW>(batch, ctas_per_sm);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D>
+template <int D, bool NARROW>
 void launch_tc(const DecodeParams& p, int hpc, int grid, cudaStream_t s) {
   switch (hpc) {
-    case 1: decode_tc_kernel<D, 1><<<grid, 32, tc_smem_bytes<D, 1>(p.B), s>>>(p); break;
-    case 2: decode_tc_kernel<D, 2><<<grid, 64, tc_smem_bytes<D, 2>(p.B), s>>>(p); break;
-    default: decode_tc_kernel<D, 4><<<grid, 128, tc_smem_bytes<D, 4>(p.B), s>>>(p); break;
+    case 1: decode_tc_kernel<D, 1, NARROW><<<grid, 32, tc_smem_bytes<D, 1>(p.B), s>>>(p); break;
+    case 2: decode_tc_kernel<D, 2, NARROW><<<grid, 64, tc_smem_bytes<D, 2>(p.B), s>>>(p); break;
+    default: decode_tc_kernel<D, 4, NARROW><<<grid, 128, tc_smem_bytes<D, 4>(p.B), s>>>(p); break;
   }
 }
 
@@ -1258,17 +1340,18 @@ bool tc_supported(int batch, int hkv, int max_pages) {
 // KV heads per CTA: the largest of 4, 2, 1 that divides Hkv.
 int tc_heads_per_cta(int hkv) { return hkv % 4 == 0 ? 4 : (hkv % 2 == 0 ? 2 : 1); }
 
-cudaError_t tc_grid(int batch, int d, int hkv, int* grid) {
+cudaError_t tc_grid(int batch, int d, int hq, int hkv, int* grid) {
   int dev = 0, sms = 0, per = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const int hpc = tc_heads_per_cta(hkv);
+  const bool narrow = hq / hkv <= 4;
   switch (d) {
-    case 64: e = tc_occupancy_hpc<64>(hpc, batch, &per); break;
-    case 128: e = tc_occupancy_hpc<128>(hpc, batch, &per); break;
-    case 256: e = tc_occupancy_hpc<256>(hpc, batch, &per); break;
+    case 64: e = narrow ? tc_occupancy_hpc<64, true>(hpc, batch, &per) : tc_occupancy_hpc<64, false>(hpc, batch, &per); break;
+    case 128: e = narrow ? tc_occupancy_hpc<128, true>(hpc, batch, &per) : tc_occupancy_hpc<128, false>(hpc, batch, &per); break;
+    case 256: e = narrow ? tc_occupancy_hpc<256, true>(hpc, batch, &per) : tc_occupancy_hpc<256, false>(hpc, batch, &per); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
@@ -1280,10 +1363,11 @@ int tc_warps_per_cta(int hkv) { return tc_heads_per_cta(hkv); }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s) {
   const int hpc = tc_heads_per_cta(p.Hkv);
+  const bool narrow = p.G <= 4;
   switch (head_dim) {
-    case 64: launch_tc<64>(p, hpc, grid, s); break;
-    case 128: launch_tc<128>(p, hpc, grid, s); break;
-    case 256: launch_tc<256>(p, hpc, grid, s); break;
+    case 64: narrow ? launch_tc<64, true>(p, hpc, grid, s) : launch_tc<64, false>(p, hpc, grid, s); break;
+    case 128: narrow ? launch_tc<128, true>(p, hpc, grid, s) : launch_tc<128, false>(p, hpc, grid, s); break;
+    case 256: narrow ? launch_tc<256, true>(p, hpc, grid, s) : launch_tc<256, false>(p, hpc, grid, s); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -45,7 +45,7 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
     // persistent grid, every warp a stream-K worker; one partial state per
     // (warp, pair) boundary: at most warps + pairs records
     int grid = 0;
-    cudaError_t e = tc_grid(batch, d, hkv, &grid);
+    cudaError_t e = tc_grid(batch, d, hq, hkv, &grid);
     if (e != cudaSuccess) return e;
     plan->tensor_cores = true;
     plan->grid = grid;

@@ -76,7 +76,7 @@ cudaError_t launch_decode_simple(const DecodeParams& p, int head_dim, cudaStream
 
 // tensor-core kernel (decode_tc.cu)
 bool tc_supported(int batch, int hkv, int max_pages);
-cudaError_t tc_grid(int batch, int d, int hkv, int* grid);
+cudaError_t tc_grid(int batch, int d, int hq, int hkv, int* grid);
 int tc_warps_per_cta(int hkv);
 cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s);
 
