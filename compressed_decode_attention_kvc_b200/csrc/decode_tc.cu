@@ -60,13 +60,15 @@ constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per try
 constexpr uint32_t kSpinLimit = 4000;       // ... for at most ~4 s
 constexpr int kSkip = 3;             // entry carrying an unusable page (flagged, no data)
 constexpr unsigned kFull = 0xffffffffu;
-// Work weights of one page of one KV head: the warp time it costs relative to
-// a ternary page (measured on B200: unpacking and the per-entry issue work
-// make a page's time grow more slowly than its bytes).  kCostBf16 is the
-// largest weight (it bounds the weight arithmetic).
-constexpr int kCostTern = 1, kCostFp8 = 4, kCostBf16 = 7;
-template <int D>
-__host__ __device__ constexpr int cost_bf16() { return D == 256 ? 7 : 6; }
+// Work weights of one page of one KV head, in quarters of a ternary page: the
+// time a page costs a warp (measured on B200; unpacking, the tensor-core
+// work per byte and the per-entry issue work make a page's time grow more
+// slowly than its bytes).  kCostMax bounds every weight.
+constexpr int kCostTern = 4, kCostMax = 24;
+template <int D, bool NARROW>
+__host__ __device__ constexpr int cost_hp(int fmt) {
+  return fmt == KVC_FMT_BF16 ? (D == 256 ? 21 : (NARROW ? 19 : 22)) : 9;
+}
 
 struct Desc {
   int fmt, np, bg, nrows;            // nrows: valid token rows of the entry's last page
@@ -225,18 +227,18 @@ __device__ __forceinline__ SeqShape seq_shape(int L, int sink, int window, int w
   s.cost = whp * (s.ns + (s.np - s.jw2)) + (s.jw2 - s.ns) * kCostTern;
   return s;
 }
-// weighted start of page j inside one (sequence, KV head)
+// weighted start of page j inside one (sequence, KV head group)
 __device__ __forceinline__ int cost_of_page(const SeqShape& s, int j, int whp) {
   if (j <= s.ns) return whp * j;
-  if (j <= s.jw2) return whp * s.ns + (j - s.ns);
-  return whp * s.ns + (s.jw2 - s.ns) + whp * (j - s.jw2);
+  if (j <= s.jw2) return whp * s.ns + kCostTern * (j - s.ns);
+  return whp * s.ns + kCostTern * (s.jw2 - s.ns) + whp * (j - s.jw2);
 }
 // first page whose weighted start is >= c (np when none)
 __device__ __forceinline__ int page_of_cost(const SeqShape& s, int c, int whp) {
   const int a = whp * s.ns;
   if (c <= a) return (c + whp - 1) / whp;
-  const int bnd = a + (s.jw2 - s.ns);
-  if (c <= bnd) return s.ns + (c - a);
+  const int bnd = a + kCostTern * (s.jw2 - s.ns);
+  if (c <= bnd) return s.ns + (c - a + kCostTern - 1) / kCostTern;
   return min(s.np, s.jw2 + (c - bnd + whp - 1) / whp);
 }
 
@@ -1202,7 +1204,7 @@ __global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
   int* seqC = seqP + (p.B + 1);
   int* seqL = seqC + (p.B + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int whp = p.hp == KVC_FMT_BF16 ? cost_bf16<D>() : kCostFp8;
+  const int whp = cost_hp<D, NARROW>(p.hp);
   const int nq = p.Hkv / HPC;          // head groups per sequence
 
   if (threadIdx.x < kEntries) {
@@ -1260,7 +1262,7 @@ __global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
   if (pr.U == 0) return;
   // every worker's weight range is at least twice the heaviest unit, so
   // each one owns at least one unit
-  const long long most = pr.C / (2 * kCostBf16);
+  const long long most = pr.C / (2 * kCostMax);
   pr.nwg = (int)((long long)gridDim.x < most ? gridDim.x : (most > 0 ? most : 1));
   const int W = blockIdx.x;
   if (W >= pr.nwg) return;
@@ -1334,7 +1336,7 @@ void launch_tc(const DecodeParams& p, int hpc, int grid, cudaStream_t s) {
 constexpr int kTcMaxBatch = kTcMaxBatchTpl;
 
 bool tc_supported(int batch, int hkv, int max_pages) {
-  return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages * kCostBf16 < (1ll << 31);
+  return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages * kCostMax < (1ll << 31);
 }
 
 // KV heads per CTA: the largest of 4, 2, 1 that divides Hkv.

@@ -53,47 +53,65 @@ __device__ __forceinline__ uint32_t tern_word16(const uint4& v, float t) {
   return out;
 }
 
-// One warp per (page, head) group of 16*D bf16 values = 2*D chunks of 16 B.
-// Lane l owns chunks l, l+32, ...: every load and store instruction of the
-// warp is contiguous.  gamma is a pairwise tree (per chunk, across the lane's
-// chunks, then a butterfly across lanes): depth log2(16*D) <= 12, so its
-// float32 relative error stays below 12 * 2^-24.
+// One warp per (page, head) group of 16*D bf16 values = 2*D chunks of 16 B;
+// at head_dim 256 two warps share a group (each holds 4 KB in registers, so
+// enough warps stay resident to keep HBM busy) and add their partial sums
+// through shared memory.  Lane l owns chunks l, l+32, ... of its warp's part:
+// every load and store instruction of the warp is contiguous.  gamma is a
+// pairwise tree (per chunk, across the lane's chunks, across lanes, across the
+// two parts): depth log2(16*D) <= 12, so its float32 relative error stays
+// below 12 * 2^-24.
 template <int D>
 __global__ void __launch_bounds__(256) quant_ternary_kernel(const uint4* __restrict__ src,
                                                             const int32_t* __restrict__ page_ids,
                                                             long long n_groups, int hkv,
                                                             uint16_t* __restrict__ dst,
                                                             float* __restrict__ gamma) {
-  constexpr int NC = D / 16;  // chunks per lane
-  const int lane = threadIdx.x & 31;
-  const long long grp = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (grp >= n_groups) return;
-  const long long i = grp / hkv;
-  const int h = (int)(grp - i * hkv);
-  const long long sp = page_ids ? (long long)page_ids[i] : i;
-  const uint4* s = src + (sp * hkv + h) * (2 * D);
+  constexpr int WPG = D > 128 ? 2 : 1;      // warps per group
+  constexpr int NC = D / 16 / WPG;          // chunks per lane
+  __shared__ float red[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int part = warp % WPG;
+  const long long grp = (long long)blockIdx.x * (8 / WPG) + warp / WPG;
+  const bool valid = grp < n_groups;
+  const uint4* s = src;
+  if (valid) {
+    const long long i = grp / hkv;
+    const int h = (int)(grp - i * hkv);
+    const long long sp = page_ids ? (long long)page_ids[i] : i;
+    s = src + (sp * hkv + h) * (2 * D) + part * (NC * 32);
+  }
 
   uint4 v[NC];
+  float sum = 0.f;
+  if (valid) {
 #pragma unroll
-  for (int c = 0; c < NC; ++c) v[c] = ld_stream(s + c * 32 + lane);
-
-  float part[NC];
+    for (int c = 0; c < NC; ++c) v[c] = ld_stream(s + c * 32 + lane);
+    float pt[NC];
 #pragma unroll
-  for (int c = 0; c < NC; ++c) part[c] = abs_sum8(v[c]);
+    for (int c = 0; c < NC; ++c) pt[c] = abs_sum8(v[c]);
 #pragma unroll
-  for (int w = 1; w < NC; w <<= 1)
+    for (int w = 1; w < NC; w <<= 1)
 #pragma unroll
-    for (int c = 0; c + w < NC; c += 2 * w) part[c] += part[c + w];
-  float sum = part[0];
+      for (int c = 0; c + w < NC; c += 2 * w) pt[c] += pt[c + w];
+    sum = pt[0];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    for (int o = 1; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  if constexpr (WPG > 1) {
+    if (lane == 0) red[warp] = sum;
+    __syncthreads();
+    const int w0 = warp - part;
+    sum = red[w0] + red[w0 + 1];              // same order in both warps
+  }
+  if (!valid) return;
 
   const float g = sum * (1.0f / (16 * D));  // exact: a power of two
   const float t = 0.5f * g;
-  uint16_t* out = dst + grp * (2 * D);      // 4*D bytes per group
+  uint16_t* out = dst + grp * (2 * D) + part * (NC * 32);   // 4*D bytes per group
 #pragma unroll
   for (int c = 0; c < NC; ++c) out[c * 32 + lane] = (uint16_t)tern_word16(v[c], t);
-  if (lane == 0) gamma[grp] = g;
+  if (lane == 0 && part == 0) gamma[grp] = g;
 }
 
 // One CTA per page: amax over the whole page (all heads), then
@@ -228,7 +246,7 @@ int grid_for(long long work, int per_block) {
 cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, int n, int hkv, int d,
                                  void* dst, float* gamma, cudaStream_t s) {
   const long long groups = (long long)n * hkv;
-  const int grid = grid_for(groups, 8);
+  const int grid = grid_for(groups, d > 128 ? 4 : 8);      // groups per 256-thread CTA
   auto* in = static_cast<const uint4*>(src);
   auto* out = static_cast<uint16_t*>(dst);
   switch (d) {
