@@ -45,6 +45,7 @@ WORKLOAD_TEXT = {
     "qwen3b": "Qwen2.5-3B-shaped layer: B=8, Hq=16, Hkv=2, D=128, L=4096, sink 4, window 256 FP8, older pages ternary, 2% outlier channels",
     "llama8b": "Llama-3-8B-shaped layer: B=32, Hq=32, Hkv=8, D=128, L=32768, sink 4, window 1024 BF16, older pages ternary, random physical page placement",
     "longctx": "long-context ragged layer: B=16, Hq=24, Hkv=4, D=256, L~U[8192,131072], sink 4, window 2048 FP8, 5% BF16 anchors, Laplace values",
+    "bulk": "bulk compress + round trip: 1 GiB of bf16 KV as 32768 pages of [8 heads][16 tokens][128], N(0,1) with 1% of entries x20; ternary quantise+pack of every page, then dequantise back to bf16",
 }
 
 
@@ -53,7 +54,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS) + ["bulk"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
@@ -366,6 +367,150 @@ def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, o
             "ms_per_step": ms / steps, "steps": steps}
 
 
+# ------------------------------------------------------- bulk workload
+
+def bulk_bytes(n, H, D):
+    """Algorithmic bytes of packing (or dequantising) n pages of H groups."""
+    return n * H * (2 * P * D + P * D // 4 + 4)
+
+
+def run_bulk(args, rank, world, dev, peak, peak_src):
+    """One step = ternary quantise+pack of every page of the 1 GiB workload,
+    then dequantise all of it back to bf16 (both directions timed)."""
+    import compressed_decode_attention_kvc_b200 as K
+    pages = synth.make_bulk_pages(seed=rank, device=dev)              # [n][H][P][D] bf16
+    n, H, _, D = pages.shape
+    codes = torch.empty((n, H, P, D // 4), dtype=torch.uint8, device=dev)
+    gamma = torch.empty((n, H), dtype=torch.float32, device=dev)
+    rt = torch.empty_like(pages)
+    stream = torch.cuda.current_stream()
+    nb = bulk_bytes(n, H, D)
+    nbytes = {"pack_ternary": nb, "dequant_ternary": nb}
+
+    def step(ev=None):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if ev is not None else None
+        if e: e[0].record(stream)
+        K.kvc_quantize_pack_pages(pages, None, n, P, H, D, K.KVC_FMT_TERNARY2, codes, gamma)
+        if e: e[1].record(stream)
+        K.kvc_dequantize_pages(codes, gamma, None, n, P, H, D, K.KVC_FMT_TERNARY2, rt)
+        if e:
+            e[2].record(stream)
+            ev.append(("pack_ternary", e[0], e[1]))
+            ev.append(("dequant_ternary", e[1], e[2]))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    marks = []
+    for _ in range(min(args.steps, 20)):
+        step(marks)
+    torch.cuda.synchronize()
+    per_kernel = {}
+    for name, e0, e1 in marks:
+        per_kernel.setdefault(name, []).append(e0.elapsed_time(e1))
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[torch.cuda.current_device()])
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    del graph
+    step_bytes = sum(nbytes.values())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    kernels = {}
+    for name, ts in per_kernel.items():
+        avg = sum(ts) / len(ts)
+        gbs = nbytes[name] / (avg * 1e-3) / 1e9
+        kernels[name] = {"ms": round(avg, 5), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                         "bytes": int(nbytes[name]), "share": 0.0}
+    tot = sum(k["ms"] for k in kernels.values())
+    for k in kernels.values():
+        k["share"] = round(k["ms"] / tot, 4)
+    dom = max(kernels, key=lambda nm: kernels[nm]["ms"])
+
+    def roof(name):
+        k = kernels[name]
+        return {"bound": "hbm", "achieved": k["gbs"], "peak": peak, "unit": "GB/s", "frac": k["frac"],
+                "traffic": ncu_traffic(name), "kernel": name, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": k["bytes"]}
+
+    res = {"value": step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9,
+           "ms_per_step": total_ms / args.steps, "kernels": kernels, "roofline": roof(dom),
+           "pack_roofline": roof("pack_ternary"), "dequant_roofline": roof("dequant_ternary"),
+           "gpu_launches": 2 * args.steps, "clocks": clk, "step_bytes": step_bytes,
+           "cfg": {"batch": n, "context": P, "n_q_heads": 0, "n_kv_heads": H, "head_dim": D},
+           "pages": {"bf16": 0, "fp8": 0, "ternary": n}}
+    if not args.no_e2e:
+        hp_src = torch.empty(pages.shape, dtype=pages.dtype, pin_memory=True)
+        hp_src.copy_(pages)
+        h_rt = torch.empty(pages.shape, dtype=pages.dtype, pin_memory=True)
+        steps = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            pages.copy_(hp_src, non_blocking=True)
+            K.kvc_quantize_pack_pages(pages, None, n, P, H, D, K.KVC_FMT_TERNARY2, codes, gamma)
+            K.kvc_dequantize_pages(codes, gamma, None, n, P, H, D, K.KVC_FMT_TERNARY2, rt)
+            h_rt.copy_(rt, non_blocking=True)
+            stream.synchronize()
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        res["e2e"] = {"value": step_bytes * world * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+                      "h2d_bytes_per_step": int(pages.numel() * 2), "d2h_bytes_per_step": int(rt.numel() * 2),
+                      "ms_per_step": ms / steps, "steps": steps}
+    return res
+
+
+def oracle_bulk_sample(n_pages=48, seed=0):
+    """Oracle work on a sample of bulk pages: pack + dequantise; returns bytes."""
+    import oracle as O
+    pages = synth.make_bulk_pages(seed=seed, device="cpu", n_pages=n_pages)
+    bits = pages.contiguous().view(torch.int16).numpy().view(np.uint16)
+    codes, gamma = O.quantize_pack_ternary(bits)
+    O.dequantize_ternary(codes, gamma)
+    n, H, _, D = pages.shape
+    return 2 * bulk_bytes(n, H, D)
+
+
 # --------------------------------------------------------- oracle arm
 
 def oracle_sample_step(inp, cfg, pairs):
@@ -409,6 +554,16 @@ def pick_pairs(cfg, inp, k, offset=0):
 
 
 def cpu_baseline(args, budget_s=12.0):
+    if args.workload == "bulk":
+        nbytes, k = 0, 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget_s:
+            nbytes += oracle_bulk_sample(seed=k)
+            k += 1
+        dt = time.perf_counter() - t0
+        return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                "sample": f"{k} x 48 pages of the bulk workload: oracle ternary pack + dequantise, "
+                          f"{dt:.1f} s on one host core"}
     inp = oracle_inputs(args.workload)
     cfg = inp["cfg"]
     pairs_done, nbytes = 0, 0
@@ -423,6 +578,20 @@ def cpu_baseline(args, budget_s=12.0):
 
 
 def run_reference(args):
+    if args.workload == "bulk":
+        for i in range(args.warmup):
+            oracle_bulk_sample(seed=i)
+        t0 = time.perf_counter()
+        nbytes = sum(oracle_bulk_sample(seed=args.warmup + i) for i in range(args.steps))
+        dt = time.perf_counter() - t0
+        v = nbytes / dt / 1e9
+        sample = "each step: 48 pages of the bulk workload - oracle ternary pack + dequantise, on one host core"
+        return {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": bulk_config_block(args),
+                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     inp = oracle_inputs(args.workload)
     cfg = inp["cfg"]
     for i in range(args.warmup):
@@ -441,6 +610,18 @@ def run_reference(args):
             "data": "synthetic", "config": config_block(args, cfg),
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def bulk_config_block(args):
+    b = synth.BULK
+    return {"workload": f"bulk: {WORKLOAD_TEXT['bulk']}", "n_pages": b["n_pages"],
+            "n_kv_heads": b["n_kv_heads"], "head_dim": b["head_dim"], "page_size": P,
+            "step": "ternary quantise+pack of all pages, then dequantise all pages to bf16",
+            "l2": "inputs larger than L2 (1 GiB of bf16 pages)",
+            "timing": ("CUDA events around K eager steps" if args.eager else
+                       "CUDA events around K replays of one captured step (CUDA graph)")
+                      + "; per-kernel times from event pairs around each launch in eager steps",
+            "parallelism": f"dp{args.gpus} (independent data per GPU)"}
 
 
 def config_block(args, cfg):
@@ -472,15 +653,16 @@ def main():
         from datetime import timedelta
         torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     peak, peak_src = load_peaks()
-    r = run_ours(args, rank, world, dev, peak, peak_src)
+    bulk = args.workload == "bulk"
+    r = (run_bulk if bulk else run_ours)(args, rank, world, dev, peak, peak_src)
     line = None
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(r["value"], 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": config_block(args, r["cfg"]),
-            "roofline": r["roofline"], "decode_roofline": r["decode_roofline"],
+            "data": "synthetic", "config": bulk_config_block(args) if bulk else config_block(args, r["cfg"]),
+            "roofline": r["roofline"], "decode_roofline": r.get("decode_roofline"),
             "kernels": r["kernels"], "pages": r["pages"], "gpu_launches": r["gpu_launches"],
             "clocks": r["clocks"], "e2e": r.get("e2e"),
         }
