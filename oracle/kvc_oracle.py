@@ -472,6 +472,95 @@ def decode_attention(q_bits, cache: PagedCache, block_table, fmt, context_lens,
 
 
 # ---------------------------------------------------------------------------
+# Append one token and retier  [Vantage, "Core architecture" (sinks kept,
+# the window slides); Minima, "Recent, Anchor and Stale" (recent pages move
+# to the compressed stale tier as they age)]
+# ---------------------------------------------------------------------------
+
+def leaving_page(context_len: int, sink: int, window: int) -> int:
+    """The page that leaves the high-precision window when token
+    ``context_len`` (0-based) is appended, or -1.  With page-granular
+    windows a page j stops being high precision when its last token
+    (j+1)*P - 1 falls below L' - window, L' = context_len + 1, i.e. when
+    (j+1)*P == context_len - window + 1; sink pages never leave."""
+    if window < 1:
+        return -1
+    x = context_len - window + 1
+    if x <= 0 or x % PAGE_SIZE:
+        return -1
+    j = x // PAGE_SIZE - 1
+    return j if j * PAGE_SIZE >= sink else -1
+
+
+def append_retier(cache: PagedCache, block_table, context_lens, k_new, v_new, tern_slot,
+                  sink: int, window: int, hp_fmt: int, older_fmt=None):
+    """One decode step's cache update, per sequence b (lengths before the
+    append; requires window >= 1, so the newest page is high precision):
+
+    1. retier: if a page j0 leaves the window (``leaving_page``) and its tag
+       is ternary (``older_fmt`` None, or older_fmt[b][j0] == TERNARY), its
+       high-precision content -- the bf16 page, or bf16(s*e) of an FP8 page --
+       is quantised to ternary (the ternary codec) into ternary-pool slot
+       tern_slot[b]; block_table[b][j0] becomes that slot and the old
+       high-precision slot is reported as freed.  A tag equal to hp_fmt keeps
+       the page where it is (an anchor).
+    2. append: token L = context_lens[b] goes to row L % P of page L // P,
+       whose high-precision slot block_table[b][L // P] the caller has set;
+       a page starting at row 0 is zeroed first.  BF16 pages take the bf16
+       row as it is; FP8 pages are re-quantised as a whole: decode every row
+       to bf16(s*e), put the new row in, quantise the page again.
+
+    k_new, v_new: bf16 bits [B][Hkv][D].  Returns (cache', block_table',
+    freed int32 [B] with -1 for none, older_fmt' or None); the inputs are not
+    modified."""
+    import copy
+    c = copy.deepcopy(cache)
+    bt = np.array(block_table, dtype=np.int32, copy=True)
+    tags = None if older_fmt is None else np.array(older_fmt, dtype=np.uint8, copy=True)
+    B = bt.shape[0]
+    freed = np.full(B, -1, dtype=np.int32)
+    k_new = np.asarray(k_new, np.uint16)
+    v_new = np.asarray(v_new, np.uint16)
+    for b in range(B):
+        L = int(context_lens[b])
+        j0 = leaving_page(L, sink, window)
+        tag = TERNARY if (tags is None or j0 < 0) else int(tags[b, j0])
+        if j0 >= 0 and tag == TERNARY:
+            phys, ts = int(bt[b, j0]), int(tern_slot[b])
+            for which in ("k", "v"):
+                if hp_fmt == BF16:
+                    page = getattr(c, which + "_bf16")[phys]
+                else:
+                    page = dequantize_fp8(getattr(c, which + "_fp8")[phys:phys + 1],
+                                          getattr(c, which + "_fp8_scale")[phys:phys + 1])[0]
+                codes, gam = quantize_pack_ternary(page[None])
+                getattr(c, which + "_tern")[ts] = codes[0]
+                getattr(c, which + "_gamma")[ts] = gam[0]
+            bt[b, j0] = ts
+            freed[b] = phys
+        j, r = L // PAGE_SIZE, L % PAGE_SIZE
+        phys = int(bt[b, j])
+        for which, new in (("k", k_new[b]), ("v", v_new[b])):
+            if hp_fmt == BF16:
+                pool = getattr(c, which + "_bf16")
+                if r == 0:
+                    pool[phys] = 0
+                pool[phys][:, r, :] = new
+            else:
+                pool = getattr(c, which + "_fp8")
+                scl = getattr(c, which + "_fp8_scale")
+                if r == 0:
+                    page = np.zeros(pool.shape[1:], dtype=np.uint16)
+                else:
+                    page = dequantize_fp8(pool[phys:phys + 1], scl[phys:phys + 1])[0]
+                page[:, r, :] = new
+                e, sc = quantize_fp8_pages(page[None])
+                pool[phys] = e[0]
+                scl[phys] = sc[0]
+    return c, bt, freed, tags
+
+
+# ---------------------------------------------------------------------------
 # Storage accounting  [Vantage, "Core architecture"; Minima, "Why the KV cache
 # becomes a bottleneck" and "What the memory measurements showed"]
 # ---------------------------------------------------------------------------

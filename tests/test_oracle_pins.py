@@ -436,3 +436,158 @@ def test_physical_placement_is_invisible():
     o2 = O.decode_attention(q, c2, bt2, f2, lens, hkv)
     assert np.abs(o1 - o2).max() < 1e-13
     assert {O.BF16, O.FP8_E4M3, O.TERNARY} <= set(np.unique(f1).tolist())
+
+
+# ------------------------------------------------------- append and retier
+
+def _pages_up_to(rng, B, max_pages, hkv, d, upto):
+    """bf16 bits [B][max_pages][Hkv][P][D]: N(0,1) for tokens < upto[b],
+    zero after (a page that is being filled has zero rows past its end)."""
+    x = rng.standard_normal((B, max_pages, hkv, O.PAGE_SIZE, d)).astype(np.float32)
+    tok = (np.arange(max_pages)[:, None] * O.PAGE_SIZE + np.arange(O.PAGE_SIZE)[None, :])
+    for b in range(B):
+        x[b][(tok >= upto[b])[:, None, :, None].repeat(hkv, 1).repeat(d, 3)] = 0.0
+    return bf16_bits(x)
+
+
+def _decoded_logical(cache, bt, fmt, lens, hkv):
+    out = {}
+    for b in range(bt.shape[0]):
+        for j in range(O.num_pages(int(lens[b]))):
+            for h in range(hkv):
+                for w in ("k", "v"):
+                    out[(b, j, h, w)] = O.decoded_page_f64(cache, w, int(fmt[b, j]), int(bt[b, j]), h)
+    return out
+
+
+def test_leaving_page_matches_page_format():
+    # the page that leaves is exactly the one whose format flips from hp to older
+    for sink, window in [(4, 64), (4, 1024), (0, 16), (40, 33), (4, 1)]:
+        for L in range(0, 400):
+            before = [O.page_format(j, L, sink, window, O.BF16, O.TERNARY) for j in range(O.num_pages(L))]
+            after = [O.page_format(j, L + 1, sink, window, O.BF16, O.TERNARY) for j in range(O.num_pages(L))]
+            flips = [j for j in range(len(before)) if before[j] == O.BF16 and after[j] == O.TERNARY]
+            j0 = O.leaving_page(L, sink, window)
+            assert flips == ([j0] if j0 >= 0 else []), (sink, window, L)
+
+
+def test_append_retier_bf16_equals_building_the_longer_cache():
+    """Appending token L to a cache built for L tokens gives the same logical
+    pages as building the cache for L + 1 tokens from scratch (BF16 window;
+    retiered pages go through the same ternary codec on the same bf16 data)."""
+    rng = np.random.default_rng(5)
+    B, max_pages, hkv, d, sink, window = 5, 9, 2, 16, 4, 40
+    # lengths hit a retier (L - window + 1 = 16k: L = 71, 87), a fresh page
+    # (L % 16 == 0: L = 64) and neither
+    lens = np.array([71, 64, 31, 87, 20], dtype=np.int32)
+    assert [O.leaving_page(int(L), sink, window) for L in lens] == [1, -1, -1, 2, -1]
+    k_full = _pages_up_to(rng, B, max_pages, hkv, d, lens + 1)
+    v_full = _pages_up_to(rng, B, max_pages, hkv, d, lens + 1)
+    k_old, v_old = k_full.copy(), v_full.copy()
+    for b, L in enumerate(lens):                      # token L not yet in the cache
+        k_old[b, L // 16, :, L % 16] = 0
+        v_old[b, L // 16, :, L % 16] = 0
+    cache, bt, fmt = O.build_paged_cache(k_old, v_old, lens, sink, window, O.BF16)
+    # the caller provides the new page's hp slot and a ternary slot for the retier
+    n_bf, n_t = cache.k_bf16.shape[0], cache.k_tern.shape[0]
+    extra = 2 * B
+    grow = lambda a, n: np.concatenate([a, np.zeros((n,) + a.shape[1:], a.dtype)])
+    cache.k_bf16, cache.v_bf16 = grow(cache.k_bf16, extra), grow(cache.v_bf16, extra)
+    cache.k_tern, cache.v_tern = grow(cache.k_tern, extra), grow(cache.v_tern, extra)
+    cache.k_gamma, cache.v_gamma = grow(cache.k_gamma, extra), grow(cache.v_gamma, extra)
+    cache.k_bf16[n_bf:] = 0x7FC0                      # stale NaN-looking slots must be zeroed
+    cache.v_bf16[n_bf:] = 0x7FC0
+    for b, L in enumerate(lens):
+        if L % 16 == 0:
+            bt[b, L // 16] = n_bf + b
+    tern_slot = n_t + np.arange(B, dtype=np.int32)
+    kn = np.stack([k_full[b, L // 16, :, L % 16] for b, L in enumerate(lens)])
+    vn = np.stack([v_full[b, L // 16, :, L % 16] for b, L in enumerate(lens)])
+    c2, bt2, freed, _ = O.append_retier(cache, bt, lens, kn, vn, tern_slot, sink, window, O.BF16)
+    fmt2 = np.full_like(fmt, 255)
+    for b in range(B):
+        for j in range(O.num_pages(int(lens[b]) + 1)):
+            fmt2[b, j] = O.page_format(j, int(lens[b]) + 1, sink, window, O.BF16, O.TERNARY)
+    ref_cache, ref_bt, ref_fmt = O.build_paged_cache(k_full, v_full, lens + 1, sink, window, O.BF16)
+    assert np.array_equal(fmt2, ref_fmt)
+    got = _decoded_logical(c2, bt2, fmt2, lens + 1, hkv)
+    ref = _decoded_logical(ref_cache, ref_bt, ref_fmt, lens + 1, hkv)
+    assert got.keys() == ref.keys()
+    for key in ref:
+        assert np.array_equal(got[key], ref[key]), key
+    for b, L in enumerate(lens):
+        j0 = O.leaving_page(int(L), sink, window)
+        assert freed[b] == (bt[b, j0] if j0 >= 0 else -1)
+        if j0 >= 0:
+            assert bt2[b, j0] == tern_slot[b]
+    # the inputs are not modified
+    assert np.array_equal(cache.k_bf16[n_bf:], np.full_like(cache.k_bf16[n_bf:], 0x7FC0))
+
+
+def test_append_retier_fp8_rows_and_untouched_codes():
+    """FP8 window: the new row decodes to the new values within e4m3 rounding,
+    rows past it stay zero, and when the new row does not raise the page's
+    amax the codes of the other rows are unchanged (re-encoding bf16(s*e)
+    with the same scale returns e); a fresh page starts from zeros."""
+    rng = np.random.default_rng(9)
+    hkv, d, sink, window = 2, 32, 4, 64
+    L = 37                                             # row 5 of page 2
+    k = _pages_up_to(rng, 1, 4, hkv, d, [L])
+    v = _pages_up_to(rng, 1, 4, hkv, d, [L])
+    cache, bt, fmt = O.build_paged_cache(k, v, [L], sink, window, O.FP8_E4M3)
+    phys = int(bt[0, 2])
+    small = bf16_bits(0.25 * np.clip(rng.standard_normal((1, hkv, d)), -1, 1))   # below amax
+    c2, bt2, freed, _ = O.append_retier(cache, bt, [L], small, small, [0], sink, window, O.FP8_E4M3)
+    assert freed[0] == -1 and np.array_equal(bt2, bt)
+    old, new = cache.k_fp8[phys], c2.k_fp8[phys]
+    assert c2.k_fp8_scale[phys] == cache.k_fp8_scale[phys]
+    rows = [r for r in range(16) if r != 5]
+    assert np.array_equal(old[:, rows], new[:, rows])
+    dec = c2.k_fp8_scale[phys] * O.e4m3_to_f64(new[:, 5])
+    x = O.bf16_to_f64(small[0])
+    assert np.all(np.abs(dec - x) <= np.abs(x) * 2.0 ** -4 + c2.k_fp8_scale[phys] * 2.0 ** -10)
+    # a larger row raises amax and the scale
+    big = bf16_bits(8.0 * np.ones((1, hkv, d)))
+    c3, _, _, _ = O.append_retier(cache, bt, [L], big, big, [0], sink, window, O.FP8_E4M3)
+    assert c3.v_fp8_scale[phys] == np.float32(8.0 / 448.0)
+    assert np.all(O.e4m3_to_f64(c3.v_fp8[phys][:, 5]) == 448.0)
+    # fresh page: everything but the new row is zero
+    L2 = 48
+    k2 = _pages_up_to(rng, 1, 4, hkv, d, [L2])
+    cache2, bt2b, _ = O.build_paged_cache(k2, k2, [L2], sink, window, O.FP8_E4M3)
+    cache2.k_fp8 = np.concatenate([cache2.k_fp8, np.full((1, hkv, 16, d), 0x55, np.uint8)])
+    cache2.v_fp8 = np.concatenate([cache2.v_fp8, np.full((1, hkv, 16, d), 0x55, np.uint8)])
+    cache2.k_fp8_scale = np.concatenate([cache2.k_fp8_scale, np.float32([3.0])])
+    cache2.v_fp8_scale = np.concatenate([cache2.v_fp8_scale, np.float32([3.0])])
+    bt2b[0, 3] = cache2.k_fp8.shape[0] - 1
+    c4, _, _, _ = O.append_retier(cache2, bt2b, [L2], small, small, [0], sink, window, O.FP8_E4M3)
+    pg = c4.k_fp8[-1]
+    assert np.all(pg[:, 1:] == 0) and np.any(pg[:, 0] != 0)
+
+
+def test_append_retier_keeps_sinks_and_anchors():
+    rng = np.random.default_rng(3)
+    hkv, d = 1, 8
+    # window 16: at L = 47, page 1 (tokens 16..31) leaves -- unless it holds
+    # sink tokens (sink 20); page 0 always holds sink tokens
+    assert O.leaving_page(47, 20, 16) == -1
+    assert O.leaving_page(47, 4, 16) == 1
+    assert O.leaving_page(31, 4, 16) == -1
+    L = 31
+    k = _pages_up_to(rng, 1, 3, hkv, d, [L])
+    cache, bt, fmt = O.build_paged_cache(k, k, [L], 4, 16, O.BF16)
+    # a page tagged as a BF16 anchor stays where it is
+    tags = np.full((1, 3), O.TERNARY, np.uint8)
+    tags[0, 1] = O.BF16
+    L3 = 47                                            # page 1 leaves
+    k3 = _pages_up_to(rng, 1, 3, hkv, d, [L3])
+    c3, bt3, _ = O.build_paged_cache(k3, k3, [L3], 4, 16, O.BF16)
+    assert c3.k_tern.shape[0] == 0                     # room for the retiered page
+    for w in ("k", "v"):
+        setattr(c3, w + "_tern", np.zeros((1, hkv, 16, d // 4), np.uint8))
+        setattr(c3, w + "_gamma", np.zeros((1, hkv), np.float32))
+    nz = bf16_bits(np.ones((1, hkv, d)))
+    out, bt_out, freed, tags_out = O.append_retier(c3, bt3, [L3], nz, nz, [0], 4, 16, O.BF16, older_fmt=tags)
+    assert freed[0] == -1 and bt_out[0, 1] == bt3[0, 1]
+    out2, bt_out2, freed2, _ = O.append_retier(c3, bt3, [L3], nz, nz, [0], 4, 16, O.BF16)
+    assert freed2[0] == bt3[0, 1] and bt_out2[0, 1] == 0
