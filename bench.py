@@ -301,10 +301,87 @@ def run_ours(args, rank, world, dev, peak, peak_src):
         "pages": {"bf16": layout.pool_pages[0], "fp8": layout.pool_pages[1], "ternary": layout.pool_pages[2]},
     }
 
+    ap = time_append_retier(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp, peak)
+    if ap is not None:
+        res["kernels"]["append_retier"] = ap
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out,
                              step_bytes, world, dev, hp)
     return res
+
+
+def time_append_retier(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp, peak):
+    """The next row of the design: one decode step's cache update
+    (kvc_append_retier) on this batch, timed alone and not part of the step.
+    Each sequence appends token L - 1 of a length-(L - 1) cache, so the page
+    leaving the window is retiered for every sequence whose L - window is a
+    multiple of 16; a scratch copy of the block table is restored before
+    each call, and retiered pages overwrite ternary slots 0..B-1 (timing
+    only; the step above has already been measured)."""
+    if cfg["window"] < 1:
+        return None
+    dev = lens.device
+    lens_a = (lens - 1).clamp(min=0)
+    bt0 = cache.block_table.clone()
+    # the cache holds L tokens, so the page leaving the window at length
+    # L - 1 is already ternary: give it the high-precision slot of another
+    # window page (not the newest) so the retier reads a valid page
+    for b, L in enumerate(lens_a.cpu().tolist()):
+        x = L - cfg["window"] + 1
+        if x > 0 and x % P == 0 and (x // P - 1) * P >= cfg["sink"] and L // P >= 1:
+            bt0[b, x // P - 1] = cache.block_table[b, L // P - 1]
+    bt = bt0.clone()
+    n_t = cache.struct.n_pages[2]
+    if n_t < B:
+        return None
+    tern_slot = torch.arange(B, dtype=torch.int32, device=dev)
+    freed = torch.empty(B, dtype=torch.int32, device=dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    k_new = torch.randn((B, H, D), device=dev).to(torch.bfloat16)
+    v_new = torch.randn((B, H, D), device=dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def one():
+        bt.copy_(bt0)
+        K.kvc_append_retier(k_new, v_new, cache.struct, bt, None, lens_a, tern_slot, freed, flags, B, H, D,
+                            P, max_pages, cfg["sink"], cfg["window"], hp)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    if int(flags.item()):
+        raise RuntimeError(f"append_retier device flags {int(flags.item())}")
+    n_ret = int((freed >= 0).sum().item())
+    # device time: replay a captured graph of reps (restore + append) pairs,
+    # minus the same graph with the restore copies alone
+    reps = 20
+    g_full, g_copy = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_full):
+        for _ in range(reps):
+            one()
+    with torch.cuda.graph(g_copy):
+        for _ in range(reps):
+            bt.copy_(bt0)
+    times = []
+    for g in (g_full, g_copy):
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / (5 * reps))
+    del g_full, g_copy
+    ms = max(times[0] - times[1], 1e-6)
+    row = 2 * H * D * 2
+    page = 2 * H * P * D * (2 if hp == K.KVC_FMT_BF16 else 1)
+    nbytes = B * 2 * row + (0 if hp == K.KVC_FMT_BF16 else B * 2 * page) + n_ret * (page + 2 * H * (P * D // 4 + 4) + 8)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes": int(nbytes),
+            "share": None, "sequences_retiered": n_ret, "note": "one decode step's append + retier, not in the step"}
 
 
 def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out, step_bytes,

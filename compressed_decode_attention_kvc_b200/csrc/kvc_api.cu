@@ -130,6 +130,37 @@ kvc_status kvc_dequantize_pages(const void* src, const float* src_scale, const i
   }
 }
 
+kvc_status kvc_append_retier(const void* k_new_bf16, const void* v_new_bf16,
+                             const kvc_paged_cache* cache, int32_t* block_table, uint8_t* older_fmt,
+                             const int32_t* context_lens, const int32_t* ternary_slot,
+                             int32_t* freed_hp_slot, uint32_t* device_flags, int batch, int n_kv_heads,
+                             int head_dim, int page_size, int max_pages, int sink_tokens,
+                             int window_tokens, kvc_format hp_mode, kvc_stream_t stream) {
+  if (batch < 0 || n_kv_heads < 1 || max_pages < 1 || sink_tokens < 0 || window_tokens < 1)
+    return KVC_ERR_INVALID_ARG;
+  if (page_size != KVC_PAGE_SIZE || !head_dim_ok(head_dim)) return KVC_ERR_UNSUPPORTED;
+  if (hp_mode != KVC_FMT_BF16 && hp_mode != KVC_FMT_FP8_E4M3) return KVC_ERR_INVALID_ARG;
+  if (!cache) return KVC_ERR_INVALID_ARG;
+  if (batch == 0) return KVC_OK;
+  if (!k_new_bf16 || !v_new_bf16 || !block_table || !context_lens || !ternary_slot || !freed_hp_slot)
+    return KVC_ERR_INVALID_ARG;
+  if (!aligned(k_new_bf16, 16) || !aligned(v_new_bf16, 16)) return KVC_ERR_INVALID_ARG;
+  const bool bf = hp_mode == KVC_FMT_BF16;
+  const void* hk = bf ? cache->k_bf16 : cache->k_fp8;
+  const void* hv = bf ? cache->v_bf16 : cache->v_fp8;
+  if (!hk || !hv || !aligned(hk, 16) || !aligned(hv, 16)) return KVC_ERR_INVALID_ARG;
+  if (!bf && (!cache->k_fp8_scale || !cache->v_fp8_scale)) return KVC_ERR_INVALID_ARG;
+  if (cache->n_pages[2] > 0 &&
+      (!cache->k_tern || !cache->v_tern || !cache->k_gamma || !cache->v_gamma ||
+       !aligned(cache->k_tern, 16) || !aligned(cache->v_tern, 16)))
+    return KVC_ERR_INVALID_ARG;
+  return from_cuda(kvc::launch_append_retier(k_new_bf16, v_new_bf16, *cache, block_table, older_fmt,
+                                             context_lens, ternary_slot, freed_hp_slot, device_flags,
+                                             batch, n_kv_heads, head_dim, max_pages, sink_tokens,
+                                             window_tokens, hp_mode,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvc_status kvc_plan_paged_cache(const int32_t* context_lens, int batch, int max_pages,
                                 int page_size, int sink_tokens, int window_tokens,
                                 kvc_format hp_mode, const uint8_t* older_fmt,

@@ -235,6 +235,225 @@ __global__ void __launch_bounds__(256) dequant_fp8_kernel(const uint2* __restric
   }
 }
 
+// --------------------------------------------------------- append + retier
+// One decode step's cache update, one CTA per sequence b (length L before
+// the step; Vantage's sinks stay and the recent window slides, "Core
+// architecture"; Minima's recent pages age into the stale tier, "Recent,
+// Anchor and Stale"):
+//   1. the page j0 that leaves the high-precision window (page-granular:
+//      (j0+1)*16 == L - window + 1, never a sink page) and is tagged ternary
+//      is quantised to ternary into slot ternary_slot[b] -- from its bf16
+//      values, or bf16(s*e) of an FP8 page -- by the same codec as the pack
+//      kernel; the block-table entry moves to that slot, the old slot is
+//      reported in freed[b];
+//   2. token L goes to row L % 16 of page L / 16 (its high-precision slot
+//      already in the block table); a page starting at row 0 is zeroed
+//      first; FP8 pages are re-quantised as a whole (decode, new row, new
+//      amax and scale, encode), in two passes that read the page from L2.
+struct AppendParams {
+  const uint16_t* k_new;      // [B][Hkv][D] bf16 bits
+  const uint16_t* v_new;
+  kvc_paged_cache cache;
+  int32_t* block_table;       // [B][max_pages]
+  uint8_t* older_fmt;         // [B][max_pages] or null
+  const int32_t* ctx;         // [B] lengths before the step
+  const int32_t* tern_slot;   // [B]
+  int32_t* freed;             // [B] out
+  uint32_t* flags;            // device error word or null
+  int Hkv, max_pages, sink, window, hp;
+};
+
+__device__ __forceinline__ void set_flag(const AppendParams& p, uint32_t f) {
+  if (p.flags) atomicOr(p.flags, f);
+}
+
+// 8 e4m3 bytes -> 8 bf16 of bf16(RN(fl32(s * e))), packed like a 16-byte chunk of bf16.
+__device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 e, float s) {
+  const uint32_t ew[2] = {e.x, e.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(ew[k >> 1] >> (16 * (k & 1)));
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(s, f.x)));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(s, f.y)));
+    o[k] = lo | (hi << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Ternary codec of one (page, head) group whose bf16 values come from an
+// hp page (BF16 pool, or FP8 pool with scale s): one warp, the same pairwise
+// tree as quant_ternary_kernel.
+template <int D>
+__device__ void retier_group(const void* hp_pool, float s, bool fp8, long long src_grp,
+                             uint16_t* tern, float* gamma, long long dst_grp, int lane) {
+  constexpr int NC = D / 16;
+  uint4 v[NC];
+  if (fp8) {
+    const uint2* src = static_cast<const uint2*>(hp_pool) + src_grp * (2 * D);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) v[c] = fp8x8_to_bf16x8(src[c * 32 + lane], s);
+  } else {
+    const uint4* src = static_cast<const uint4*>(hp_pool) + src_grp * (2 * D);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) v[c] = src[c * 32 + lane];
+  }
+  float pt[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) pt[c] = abs_sum8(v[c]);
+#pragma unroll
+  for (int w = 1; w < NC; w <<= 1)
+#pragma unroll
+    for (int c = 0; c + w < NC; c += 2 * w) pt[c] += pt[c + w];
+  float sum = pt[0];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float g = sum * (1.0f / (16 * D));
+  const float t = 0.5f * g;
+  uint16_t* out = tern + dst_grp * (2 * D);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) out[c * 32 + lane] = (uint16_t)tern_word16(v[c], t);
+  if (lane == 0) gamma[dst_grp] = g;
+}
+
+// Page value chunk c (8 bf16) after the append: the new row, zero (fresh
+// page) or the page's own value.
+template <int D>
+__device__ __forceinline__ uint4 page_chunk_after(const AppendParams& p, const uint16_t* nw, long long b,
+                                                  const void* pool, long long page, float s_old,
+                                                  int r, int c) {
+  constexpr int CPR = D / 8;                      // chunks per row
+  const int h = c / (16 * CPR), rem = c - h * 16 * CPR, row = rem / CPR, dc = rem - row * CPR;
+  if (row == r)
+    return reinterpret_cast<const uint4*>(nw)[(b * p.Hkv + h) * CPR + dc];
+  if (r == 0) return make_uint4(0u, 0u, 0u, 0u);
+  if (p.hp == KVC_FMT_FP8_E4M3)
+    return fp8x8_to_bf16x8(static_cast<const uint2*>(pool)[page * p.Hkv * 16 * CPR + c], s_old);
+  return static_cast<const uint4*>(pool)[page * p.Hkv * 16 * CPR + c];
+}
+
+template <int D>
+__device__ void append_one(const AppendParams& p, const uint16_t* nw, long long b, void* pool, float* scale,
+                           long long page, int r, float* red) {
+  constexpr int CPR = D / 8;
+  const int nchunks = p.Hkv * 16 * CPR;
+  if (p.hp == KVC_FMT_BF16) {
+    uint4* dst = static_cast<uint4*>(pool) + page * nchunks;
+    for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+      const int row = (c % (16 * CPR)) / CPR;
+      if (row == r || r == 0) dst[c] = page_chunk_after<D>(p, nw, b, pool, page, 0.f, r, c);
+    }
+    return;
+  }
+  // FP8: pass 1 -- amax of the page after the append
+  const float s_old = scale[page];
+  float amax = 0.f;
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    const uint4 v = page_chunk_after<D>(p, nw, b, pool, page, s_old, r, c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+  for (int k = 1; k < (int)(blockDim.x >> 5); ++k) amax = fmaxf(amax, red[k]);
+  __syncthreads();                                 // red is reused; every read of pass 1 is done
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  // pass 2 -- each thread re-reads and rewrites only its own chunks
+  uint2* dst = static_cast<uint2*>(pool) + page * nchunks;
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+    const uint4 v = page_chunk_after<D>(p, nw, b, pool, page, s_old, r, c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 y = make_float2(__fmul_rn(bf16_lo(w[k]), inv), __fmul_rn(bf16_hi(w[k]), inv));
+      const uint32_t e2 = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+      packed[k >> 1] |= e2 << (16 * (k & 1));
+    }
+    dst[c] = make_uint2(packed[0], packed[1]);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) scale[page] = sc;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) append_retier_kernel(AppendParams p) {
+  __shared__ float red[8];
+  const long long b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = p.ctx[b];
+  if (L < 0 || L >= p.max_pages * kPage) {
+    if (threadIdx.x == 0) {
+      set_flag(p, kErrContext);
+      p.freed[b] = -1;
+    }
+    return;
+  }
+  const long long hp_pages = p.hp == KVC_FMT_BF16 ? p.cache.n_pages[0] : p.cache.n_pages[1];
+  void* k_hp = const_cast<void*>(p.hp == KVC_FMT_BF16 ? p.cache.k_bf16 : p.cache.k_fp8);
+  void* v_hp = const_cast<void*>(p.hp == KVC_FMT_BF16 ? p.cache.v_bf16 : p.cache.v_fp8);
+  float* k_sc = const_cast<float*>(p.cache.k_fp8_scale);
+  float* v_sc = const_cast<float*>(p.cache.v_fp8_scale);
+
+  // 1. retier the page that leaves the window
+  int j0 = -1;
+  if (p.window >= 1) {
+    const int x = L - p.window + 1;
+    if (x > 0 && x % kPage == 0 && (x / kPage - 1) * kPage >= p.sink) j0 = x / kPage - 1;
+  }
+  int freed = -1, ts = -1;
+  if (j0 >= 0) {
+    const long long row = b * p.max_pages + j0;
+    const int tag = p.older_fmt ? (int)p.older_fmt[row] : KVC_FMT_TERNARY2;
+    const int phys = p.block_table[row];
+    ts = p.tern_slot[b];
+    if (tag == KVC_FMT_TERNARY2) {
+      if (phys < 0 || phys >= hp_pages || ts < 0 || ts >= p.cache.n_pages[2]) {
+        if (threadIdx.x == 0) set_flag(p, kErrBlockTable);
+      } else {
+        const bool fp8 = p.hp == KVC_FMT_FP8_E4M3;
+        for (int g = warp; g < 2 * p.Hkv; g += (int)(blockDim.x >> 5)) {
+          const bool is_v = g >= p.Hkv;
+          const int h = is_v ? g - p.Hkv : g;
+          retier_group<D>(is_v ? v_hp : k_hp, fp8 ? (is_v ? v_sc : k_sc)[phys] : 0.f, fp8,
+                          (long long)phys * p.Hkv + h,
+                          static_cast<uint16_t*>(const_cast<void*>(is_v ? p.cache.v_tern : p.cache.k_tern)),
+                          const_cast<float*>(is_v ? p.cache.v_gamma : p.cache.k_gamma),
+                          (long long)ts * p.Hkv + h, lane);
+        }
+        freed = phys;
+      }
+    } else if (tag != p.hp) {
+      if (threadIdx.x == 0) set_flag(p, kErrFormat);   // an anchor in the other high-precision format
+    }
+  }
+  __syncthreads();
+
+  // 2. append token L
+  const int j = L / kPage, r = L % kPage;
+  const int physn = p.block_table[b * p.max_pages + j];
+  if (physn < 0 || physn >= hp_pages || physn == freed) {
+    if (threadIdx.x == 0) set_flag(p, kErrBlockTable);
+  } else {
+    append_one<D>(p, p.k_new, b, k_hp, k_sc, physn, r, red);
+    append_one<D>(p, p.v_new, b, v_hp, v_sc, physn, r, red);
+  }
+  if (threadIdx.x == 0) {
+    if (freed >= 0) {
+      p.block_table[b * p.max_pages + j0] = ts;
+      if (p.older_fmt) p.older_fmt[b * p.max_pages + j0] = KVC_FMT_TERNARY2;
+    }
+    p.freed[b] = freed;
+  }
+}
+
 int grid_for(long long work, int per_block) {
   long long g = (work + per_block - 1) / per_block;
   if (g > (1ll << 30)) g = 1ll << 30;
@@ -285,6 +504,35 @@ cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const in
     case 64: dequant_ternary_kernel<64><<<grid, 256, 0, s>>>(in, gamma, page_ids, groups, hkv, out); break;
     case 128: dequant_ternary_kernel<128><<<grid, 256, 0, s>>>(in, gamma, page_ids, groups, hkv, out); break;
     case 256: dequant_ternary_kernel<256><<<grid, 256, 0, s>>>(in, gamma, page_ids, groups, hkv, out); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_retier(const void* k_new, const void* v_new, const kvc_paged_cache& cache,
+                                int32_t* block_table, uint8_t* older_fmt, const int32_t* ctx,
+                                const int32_t* tern_slot, int32_t* freed, uint32_t* flags, int batch,
+                                int hkv, int d, int max_pages, int sink, int window, int hp,
+                                cudaStream_t s) {
+  AppendParams p;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.cache = cache;
+  p.block_table = block_table;
+  p.older_fmt = older_fmt;
+  p.ctx = ctx;
+  p.tern_slot = tern_slot;
+  p.freed = freed;
+  p.flags = flags;
+  p.Hkv = hkv;
+  p.max_pages = max_pages;
+  p.sink = sink;
+  p.window = window;
+  p.hp = hp;
+  switch (d) {
+    case 64: append_retier_kernel<64><<<batch, 256, 0, s>>>(p); break;
+    case 128: append_retier_kernel<128><<<batch, 256, 0, s>>>(p); break;
+    case 256: append_retier_kernel<256><<<batch, 256, 0, s>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -41,7 +41,7 @@ ERR_TIMEOUT = 8
 EXPORTS = (
     "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
-    "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc",
+    "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc", "kvc_append_retier",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -77,6 +77,9 @@ def _load() -> ctypes.CDLL:
     lib.kvc_quantize_pack_pages.argtypes = [vp, vp, i32, i32, i32, i32, st, vp, vp, vp]
     lib.kvc_dequantize_pages.restype = st
     lib.kvc_dequantize_pages.argtypes = [vp, vp, vp, i32, i32, i32, i32, st, vp, vp]
+    lib.kvc_append_retier.restype = st
+    lib.kvc_append_retier.argtypes = [vp, vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, vp, vp, vp,
+                                      i32, i32, i32, i32, i32, i32, i32, st, vp]
     lib.kvc_plan_paged_cache.restype = st
     lib.kvc_plan_paged_cache.argtypes = [vp, i32, i32, i32, i32, i32, st, vp, vp, vp, vp, vp, vp]
     lib.kvc_decode_workspace_size.restype = st
@@ -136,6 +139,20 @@ def kvc_dequantize_pages(src, src_scale, page_ids, n, page_size, n_kv_heads, hea
     _check(_lib.kvc_dequantize_pages(_ptr(src), _ptr(src_scale), _ptr(page_ids), n, page_size,
                                      n_kv_heads, head_dim, mode, _ptr(dst_bf16), _stream(stream)),
            "kvc_dequantize_pages")
+
+
+def kvc_append_retier(k_new_bf16, v_new_bf16, cache: kvc_paged_cache, block_table, older_fmt,
+                      context_lens, ternary_slot, freed_hp_slot, device_flags, batch, n_kv_heads,
+                      head_dim, page_size, max_pages, sink_tokens, window_tokens, hp_mode,
+                      stream=None) -> None:
+    """Append one token per sequence and move the page that leaves the
+    high-precision window to the ternary pool (see include/kvc.h)."""
+    _check(_lib.kvc_append_retier(_ptr(k_new_bf16), _ptr(v_new_bf16), ctypes.byref(cache),
+                                  _ptr(block_table), _ptr(older_fmt), _ptr(context_lens),
+                                  _ptr(ternary_slot), _ptr(freed_hp_slot), _ptr(device_flags), batch,
+                                  n_kv_heads, head_dim, page_size, max_pages, sink_tokens,
+                                  window_tokens, hp_mode, _stream(stream)),
+           "kvc_append_retier")
 
 
 def kvc_plan_paged_cache(context_lens, batch, max_pages, page_size, sink_tokens, window_tokens,

@@ -146,6 +146,57 @@ typedef struct kvc_paged_cache {
 } kvc_paged_cache;
 
 /*
+ * kvc_append_retier - one decode step's cache update, for every sequence of
+ * the batch: the sink tokens stay and the high-precision window slides
+ * ("Show HN: Vantage-V-AI", section "Core architecture"), and the page that
+ * ages out of the recent tier moves to the compressed stale tier (Minima-KV,
+ * section "Recent, Anchor and Stale").  Per sequence b, with L the length
+ * BEFORE the step (window_tokens >= 1, so the newest page is high
+ * precision):
+ *   1. retier: page j0 with (j0+1)*16 == L - window_tokens + 1, unless it
+ *      holds sink tokens, leaves the window.  If its tag is TERNARY2
+ *      (older_fmt NULL, or older_fmt[b][j0] == TERNARY2) its hp_mode content
+ *      (the bf16 values, or bf16(s*e) of an FP8 page) is quantised to
+ *      ternary -- the codec of kvc_quantize_pack_pages -- into ternary slot
+ *      ternary_slot[b] of the K and V pools; block_table[b][j0] becomes that
+ *      slot, older_fmt[b][j0] (if given) TERNARY2, and freed_hp_slot[b] the
+ *      released high-precision slot.  A tag equal to hp_mode keeps the page
+ *      in place (an anchor); freed_hp_slot[b] is -1 when nothing moved.
+ *   2. append: token L (k_new[b], v_new[b]) goes to row L % 16 of page
+ *      L / 16, whose hp_mode slot the caller has put in block_table[b][L/16]
+ *      (a new slot when L % 16 == 0; that page is zeroed first).  BF16 pages
+ *      take the row as it is; FP8 pages are re-quantised whole (decode to
+ *      bf16(s*e), insert the row, new amax and scale, encode).
+ * The caller then advances its lengths to L + 1.
+ *
+ *   k_new_bf16, v_new_bf16  device bf16 [batch][Hkv][D], 16-byte aligned
+ *   cache          host pointer to the pools; the hp_mode pools and the
+ *                  ternary pools are WRITTEN (the pointers are cast from
+ *                  const); hp_mode BF16 or FP8_E4M3
+ *   block_table    device int32 [batch][max_pages], read and updated
+ *   older_fmt      device uint8 [batch][max_pages] or NULL, updated
+ *   context_lens   device int32 [batch], each in [0, max_pages*16 - 1]
+ *   ternary_slot   device int32 [batch]: ternary slot for a retiered page
+ *   freed_hp_slot  device int32 [batch], out
+ *   device_flags   device uint32 word or NULL: OR-ed with 1 (a block-table
+ *                  or ternary slot outside its pool; that part is skipped),
+ *                  2 (a leaving page tagged with the other high-precision
+ *                  format; left in place), 4 (a length out of range; the
+ *                  sequence is skipped)
+ * Errors: INVALID_ARG for null or misaligned pointers, negative sizes,
+ * window_tokens < 1 or a bad hp_mode; UNSUPPORTED for page_size != 16 or a
+ * head_dim other than 64, 128, 256.  Asynchronous on `stream`; allocates
+ * nothing.
+ */
+KVC_API kvc_status kvc_append_retier(const void* k_new_bf16, const void* v_new_bf16,
+                                     const kvc_paged_cache* cache, int32_t* block_table,
+                                     uint8_t* older_fmt, const int32_t* context_lens,
+                                     const int32_t* ternary_slot, int32_t* freed_hp_slot,
+                                     uint32_t* device_flags, int batch, int n_kv_heads,
+                                     int head_dim, int page_size, int max_pages, int sink_tokens,
+                                     int window_tokens, kvc_format hp_mode, kvc_stream_t stream);
+
+/*
  * kvc_plan_paged_cache - host-side page placement (a small block manager).
  * Decides each logical page's format with the same rule the decode kernel
  * applies, and gives every page a slot in the pool of its format.

@@ -127,3 +127,26 @@ def test_planner_argument_errors():
     with pytest.raises(K.KvcError):
         K.paged_cache.plan_paged_cache(lens[:1], 4, 4, 16, K.KVC_FMT_BF16,
                                        older_fmt=torch.full((1, 4), 9, dtype=torch.uint8))
+
+
+def test_append_retier_argument_errors():
+    """Host-side validation of kvc_append_retier (no GPU work is launched)."""
+    import ctypes
+    lib = ctypes.CDLL(K.LIB_PATH)
+    lib.kvc_append_retier.restype = ctypes.c_int
+    cache = K.kvc_paged_cache()
+    vp = ctypes.c_void_p
+    def call(batch=1, hkv=2, d=128, page=16, max_pages=4, sink=4, window=16, hp=K.KVC_FMT_BF16,
+             ptr=1 << 20, cache_p=True):
+        p = vp(ptr) if ptr else None
+        return lib.kvc_append_retier(p, p, ctypes.byref(cache) if cache_p else None, p, None, p, p, p,
+                                     None, batch, hkv, d, page, max_pages, sink, window, hp, None)
+    assert call(window=0) == K.KVC_ERR_INVALID_ARG          # the newest page must be high precision
+    assert call(page=8) == K.KVC_ERR_UNSUPPORTED
+    assert call(d=96) == K.KVC_ERR_UNSUPPORTED
+    assert call(hp=K.KVC_FMT_TERNARY2) == K.KVC_ERR_INVALID_ARG
+    assert call(cache_p=False) == K.KVC_ERR_INVALID_ARG
+    assert call(batch=0) == K.KVC_OK                        # nothing to do, nothing launched
+    assert call(ptr=0) == K.KVC_ERR_INVALID_ARG
+    assert call(ptr=(1 << 20) + 8) == K.KVC_ERR_INVALID_ARG  # misaligned new-token rows
+    assert call() == K.KVC_ERR_INVALID_ARG                  # no BF16 pools in the cache
