@@ -56,6 +56,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS) + ["bulk"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=None,
+                    help="attention layers per step (default: 36 for the Qwen2.5-3B-shaped layer, "
+                         "whose model has 36, else 1); all layers are decoded in one launch")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--eager", action="store_true",
@@ -164,9 +167,21 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     import compressed_decode_attention_kvc_b200 as K
     from compressed_decode_attention_kvc_b200 import paged_cache as PC
 
+    n_layers = layers_of(args)
     inp = synth.make_decode_inputs(args.workload, seed=rank, device=dev, batch=args.batch)
     cfg = inp["cfg"]
     B, max_pages, H, _, D = inp["k_pages"].shape
+    if n_layers > 1:
+        # further layers: their own K, V and Q, the first layer's placement
+        ks, vs, qs = [inp["k_pages"]], [inp["v_pages"]], [inp["q"]]
+        for l in range(1, n_layers):
+            o = synth.make_decode_inputs(args.workload, seed=rank * 1000 + l, device=dev, batch=args.batch)
+            ks.append(o["k_pages"]); vs.append(o["v_pages"]); qs.append(o["q"])
+            del o
+        inp["k_pages"] = torch.cat(ks)
+        inp["v_pages"] = torch.cat(vs)
+        inp["q"] = torch.cat(qs)              # [layers * B][Hq][D], layer-major
+        del ks, vs, qs
     hq = cfg["n_q_heads"]
     hp = K.KVC_FMT_BF16 if cfg["hp"] == "bf16" else K.KVC_FMT_FP8_E4M3
     older = None
@@ -176,18 +191,18 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     sk = None if inp["slot_key"] is None else inp["slot_key"].cpu()
     layout = PC.plan_paged_cache(lens_h, max_pages, cfg["sink"], cfg["window"], hp,
                                  older_fmt=None if older is None else older.cpu(), slot_key=sk)
-    cache = PC.allocate_device_cache(layout, H, D, dev)
-    kf = inp["k_pages"].view(B * max_pages, H, P, D)
-    vf = inp["v_pages"].view(B * max_pages, H, P, D)
+    cache = PC.allocate_device_cache(layout, H, D, dev, n_layers=n_layers)
+    kf = inp["k_pages"].view(n_layers * B * max_pages, H, P, D)
+    vf = inp["v_pages"].view(n_layers * B * max_pages, H, P, D)
     q, lens = inp["q"], inp["context_lens"]
-    ws_bytes = K.kvc_decode_workspace_size(B, hq, H, D, max_pages)
+    ws_bytes = K.kvc_decode_workspace_size(n_layers * B, hq, H, D, max_pages)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
-    out = torch.empty((B, hq, D), dtype=torch.float32, device=dev)
-    nbytes = algorithmic_bytes(cfg, layout, B, max_pages, older is not None)
+    out = torch.empty((n_layers * B, hq, D), dtype=torch.float32, device=dev)
+    nbytes = {k: n_layers * v for k, v in algorithmic_bytes(cfg, layout, B, max_pages, older is not None).items()}
     stream = torch.cuda.current_stream()
 
-    pools = [(f, n) for f, n in zip((K.KVC_FMT_BF16, K.KVC_FMT_FP8_E4M3, K.KVC_FMT_TERNARY2),
-                                    layout.pool_pages) if n > 0]
+    pools = [(f, n * n_layers) for f, n in zip((K.KVC_FMT_BF16, K.KVC_FMT_FP8_E4M3, K.KVC_FMT_TERNARY2),
+                                               layout.pool_pages) if n > 0]
     names = {K.KVC_FMT_BF16: "pack_bf16", K.KVC_FMT_FP8_E4M3: "pack_fp8", K.KVC_FMT_TERNARY2: "pack_ternary"}
     fields = {K.KVC_FMT_BF16: ("k_bf16", "v_bf16", None, None),
               K.KVC_FMT_FP8_E4M3: ("k_fp8", "v_fp8", "k_fp8_scale", "v_fp8_scale"),
@@ -211,8 +226,9 @@ def run_ours(args, rank, world, dev, peak, peak_src):
         if ev is not None:
             e0 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        K.kvc_decode_attention_paged(q, cache.struct, cache.block_table, older, lens, B, hq, H, D, P,
-                                     max_pages, cfg["sink"], cfg["window"], hp, 0.0, out, ws, ws_bytes)
+        K.kvc_decode_attention_paged_layers(q, cache.struct, cache.block_table, older, lens, n_layers, B,
+                                            hq, H, D, P, max_pages, cfg["sink"], cfg["window"], hp, 0.0,
+                                            out, ws, ws_bytes)
         if ev is not None:
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
@@ -264,7 +280,7 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
     del graph
-    flags = K.kvc_decode_read_error(ws, B, hq, H, D, max_pages)
+    flags = K.kvc_decode_read_error(ws, n_layers * B, hq, H, D, max_pages)
     if flags:
         raise RuntimeError(f"device error flags {flags}")
 
@@ -297,16 +313,17 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     res = {
         "value": value, "ms_per_step": ms_per_step, "kernels": kernels, "roofline": roof(dom),
         "decode_roofline": roof("decode"), "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk, "step_bytes": step_bytes, "cfg": cfg,
+        "clocks": clk, "step_bytes": step_bytes, "cfg": dict(cfg, layers=n_layers),
         "pages": {"bf16": layout.pool_pages[0], "fp8": layout.pool_pages[1], "ternary": layout.pool_pages[2]},
     }
 
-    ap = time_append_retier(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp, peak)
+    ap = None if n_layers > 1 else time_append_retier(args, K, cfg, cache, lens, older, B, H, D, max_pages,
+                                                       hp, peak)
     if ap is not None:
         res["kernels"]["append_retier"] = ap
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out,
-                             step_bytes, world, dev, hp)
+                             step_bytes, world, dev, hp, n_layers)
     return res
 
 
@@ -385,11 +402,12 @@ def time_append_retier(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp,
 
 
 def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out, step_bytes,
-            world, dev, hp):
+            world, dev, hp, n_layers=1):
     """Same step through the public API with host buffers: planner on the
     host, H2D of the bf16 pages / Q / lengths / block table from pinned
     memory, pack + decode, D2H of the output, all inside the timed region."""
     B, max_pages, H, _, D = inp["k_pages"].shape
+    B //= n_layers                                   # the inputs stack the layers
     hq = cfg["n_q_heads"]
     hk = torch.empty(kf.shape, dtype=kf.dtype, pin_memory=True)
     hv = torch.empty(vf.shape, dtype=vf.dtype, pin_memory=True)
@@ -413,10 +431,14 @@ def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, o
         cache.block_table.copy_(lay.block_table.pin_memory(), non_blocking=True)
         for f in range(3):
             if lay.pool_pages[f]:
-                cache.page_ids[f].copy_(lay.pool_src_ids[f].pin_memory(), non_blocking=True)
+                ids = lay.pool_src_ids[f]
+                if n_layers > 1:
+                    ids = torch.cat([ids + l * B * max_pages for l in range(n_layers)])
+                cache.page_ids[f].copy_(ids.pin_memory(), non_blocking=True)
         PC.compress_into(cache, kf, vf)
-        K.kvc_decode_attention_paged(q_d, cache.struct, cache.block_table, older, l_d, B, hq, H, D, P,
-                                     max_pages, cfg["sink"], cfg["window"], hp, 0.0, out, ws, ws_bytes)
+        K.kvc_decode_attention_paged_layers(q_d, cache.struct, cache.block_table, older, l_d, n_layers, B,
+                                            hq, H, D, P, max_pages, cfg["sink"], cfg["window"], hp, 0.0,
+                                            out, ws, ws_bytes)
         hout.copy_(out, non_blocking=True)
         stream.synchronize()
         return float(hout[0, 0, 0])
@@ -438,7 +460,7 @@ def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, o
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     h2d = (hk.numel() * 2 + hv.numel() * 2 + hq_t.numel() * 2 + hl.numel() * 4
-           + layout.block_table.numel() * 4 + sum(len(x) for x in layout.pool_src_ids) * 4)
+           + layout.block_table.numel() * 4 + n_layers * sum(len(x) for x in layout.pool_src_ids) * 4)
     return {"value": step_bytes * world * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hout.numel() * 4),
             "ms_per_step": ms / steps, "steps": steps}
@@ -701,9 +723,19 @@ def bulk_config_block(args):
             "parallelism": f"dp{args.gpus} (independent data per GPU)"}
 
 
+def layers_of(args):
+    """Attention layers decoded per step: the Qwen2.5-3B-shaped workload runs
+    all 36 of its model's layers (one pack launch per format, one decode
+    launch for the stack); the others are one layer."""
+    return args.layers or (36 if args.workload == "qwen3b" else 1)
+
+
 def config_block(args, cfg):
     ctx = cfg["context"]
-    return {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}",
+    n_layers = layers_of(args)
+    return {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}"
+                        + (f", {n_layers} layers per step" if n_layers > 1 else ""),
+            "layers": n_layers,
             "batch": cfg["batch"], "context": list(ctx) if isinstance(ctx, tuple) else ctx,
             "n_q_heads": cfg["n_q_heads"], "n_kv_heads": cfg["n_kv_heads"], "head_dim": cfg["head_dim"],
             "page_size": P, "step": "pack every page of the batch into its format (bf16 copy / fp8 / "

@@ -69,7 +69,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_simple_kernel(DecodeParams
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G, Hkv = p.Hkv;
-  int L = p.ctx[b];
+  int L = p.ctx[b % p.Bseq];
+  const int layer = b / p.Bseq;
   if (L < 0 || L > p.max_pages * kPage) {
     if (threadIdx.x == 0) atomicOr(p.err, kErrContext);
     L = 0;
@@ -97,18 +98,19 @@ __global__ void __launch_bounds__(kWarps * 32) decode_simple_kernel(DecodeParams
   const kvc_paged_cache& c = p.cache;
 
   for (int j = j0 + warp; j < j1; j += kWarps) {
-    const long long row = (long long)b * p.max_pages + j;
+    const long long row = (long long)(b % p.Bseq) * p.max_pages + j;
     const int older = p.older_fmt ? p.older_fmt[row] : KVC_FMT_TERNARY2;
     const int fmt = page_format(j, L, p.sink, p.window, p.hp, older);
     if (fmt < 0 || fmt > 2) {
       if (lane == 0) atomicOr(p.err, kErrFormat);
       continue;
     }
-    const long long phys = p.block_table[row];
+    long long phys = p.block_table[row];
     if (phys < 0 || phys >= c.n_pages[fmt]) {
       if (lane == 0) atomicOr(p.err, kErrBlockTable);
       continue;
     }
+    phys += (long long)layer * c.n_pages[fmt];          // this layer's part of the pool
     const int nt = min(kPage, L - j * kPage);
     for (int t = 0; t < nt; ++t) {
       float kx[DPL], vx[DPL];

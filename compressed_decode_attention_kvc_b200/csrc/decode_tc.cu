@@ -296,6 +296,7 @@ __device__ __forceinline__ int meta_bg(int m) { return m >> 7; }
 
 struct MetaA {
   int phys, older, info;    // info < 0: no unit
+  int layer;                // layer of a stacked batch (pool slots offset by layer * n_pages)
 };
 struct Meta {
   int m;                    // packed fmt / ntok / bq
@@ -310,6 +311,7 @@ __device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prolog
                                              int lane, int hpc, int wi, MetaA& a) {
   a.info = -1;
   a.phys = 0;
+  a.layer = 0;
   a.older = KVC_FMT_TERNARY2;
   if (x0 >= u1) return;
   const int b0 = pr.find(pr.seqP, x0);
@@ -331,7 +333,12 @@ __device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prolog
   }
   const int g = q * hpc + wi;                      // this warp's KV head
   const int bq = b * (p.Hkv / hpc) + q;            // (sequence, head group) pair
-  const long long row = (long long)b * p.max_pages + j;
+  int rb = b;                                      // row of the shared block table
+  if (p.Bseq != p.B) {                             // stacked layers (uniform branch)
+    a.layer = b / p.Bseq;
+    rb = b - a.layer * p.Bseq;
+  }
+  const long long row = (long long)rb * p.max_pages + j;
   const int last_valid = min((j + 1) * kPage, L) - 1;
   const int is_hp = (j * kPage < p.sink || last_valid >= L - p.window) ? 1 : 0;
   a.info = min(kPage, L - j * kPage) | (is_hp << 5) | (g << 6) | (bq << 13);
@@ -356,13 +363,16 @@ __device__ __forceinline__ void meta_phase_b(const DecodeParams& p, const MetaA&
     atomicOr(p.err, kErrBlockTable);
     fmt = kSkip;
   } else {
-    m.grp = a.phys * p.Hkv + g;
+    // the layer's pool slots follow the earlier layers'
+    const int phys = a.phys + a.layer * (int)(fmt == KVC_FMT_BF16 ? p.cache.n_pages[0]
+                                             : fmt == KVC_FMT_FP8_E4M3 ? p.cache.n_pages[1] : p.cache.n_pages[2]);
+    m.grp = phys * p.Hkv + g;
     if (fmt == KVC_FMT_TERNARY2) {
       m.ks = __ldg(p.cache.k_gamma + m.grp);
       m.vs = __ldg(p.cache.v_gamma + m.grp);
     } else if (fmt == KVC_FMT_FP8_E4M3) {
-      m.ks = __ldg(p.cache.k_fp8_scale + a.phys);
-      m.vs = __ldg(p.cache.v_fp8_scale + a.phys);
+      m.ks = __ldg(p.cache.k_fp8_scale + phys);
+      m.vs = __ldg(p.cache.v_fp8_scale + phys);
     } else {
       m.ks = m.vs = 1.f;
     }
@@ -1217,7 +1227,7 @@ __global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
       const int b = base + lane;
       int u = 0, c = 0;
       if (b < p.B) {
-        int L = p.ctx[b];
+        int L = p.ctx[p.Bseq == p.B ? b : b % p.Bseq];
         if (L < 0 || L > p.max_pages * kPage) {
           if (blockIdx.x == 0) atomicOr(p.err, kErrContext);
           L = 0;

@@ -233,9 +233,25 @@ kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache*
                                       int sink_tokens, int window_tokens, kvc_format hp_mode,
                                       float softmax_scale, float* out, void* workspace,
                                       size_t workspace_bytes, kvc_stream_t stream) {
+  return kvc_decode_attention_paged_layers(q_bf16, cache, block_table, older_fmt, context_lens, 1, batch,
+                                           n_q_heads, n_kv_heads, head_dim, page_size, max_pages,
+                                           sink_tokens, window_tokens, hp_mode, softmax_scale, out,
+                                           workspace, workspace_bytes, stream);
+}
+
+kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged_cache* cache,
+                                             const int32_t* block_table, const uint8_t* older_fmt,
+                                             const int32_t* context_lens, int n_layers, int batch,
+                                             int n_q_heads, int n_kv_heads, int head_dim, int page_size,
+                                             int max_pages, int sink_tokens, int window_tokens,
+                                             kvc_format hp_mode, float softmax_scale, float* out,
+                                             void* workspace, size_t workspace_bytes, kvc_stream_t stream) {
   if (batch < 0 || max_pages < 0 || n_kv_heads < 1 || n_q_heads < 1 || sink_tokens < 0 ||
-      window_tokens < 0)
+      window_tokens < 0 || n_layers < 1)
     return KVC_ERR_INVALID_ARG;
+  if ((long long)n_layers * batch > (1ll << 30)) return KVC_ERR_INVALID_ARG;
+  const int seqs = batch;        // per layer
+  batch = n_layers * batch;      // virtual sequences (layer-major)
   if (n_q_heads % n_kv_heads) return KVC_ERR_INVALID_ARG;
   if (page_size != KVC_PAGE_SIZE || !head_dim_ok(head_dim) || n_q_heads / n_kv_heads > 8)
     return KVC_ERR_UNSUPPORTED;
@@ -269,6 +285,7 @@ kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache*
   p.older_fmt = older_fmt;
   p.ctx = context_lens;
   p.B = batch;
+  p.Bseq = seqs;
   p.Hq = n_q_heads;
   p.Hkv = n_kv_heads;
   p.G = n_q_heads / n_kv_heads;

@@ -56,6 +56,9 @@ struct DecodeParams {
   const uint8_t* older_fmt;
   const int32_t* ctx;
   int B, Hq, Hkv, G, max_pages;
+  int Bseq;                  // sequences per layer; B = layers * Bseq virtual sequences
+                             // (virtual sequence b: layer b / Bseq, sequence b % Bseq;
+                             // layer l's pool slots start at l * n_pages[format])
   int sink, window, hp;
   float scale_log2;          // softmax_scale * log2(e)
   int n_splits, pages_per_split;

@@ -42,6 +42,7 @@ EXPORTS = (
     "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
     "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc", "kvc_append_retier",
+    "kvc_decode_attention_paged_layers",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -87,6 +88,10 @@ def _load() -> ctypes.CDLL:
     lib.kvc_decode_attention_paged.restype = st
     lib.kvc_decode_attention_paged.argtypes = [
         vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, i32, i32, i32, i32, i32, i32,
+        i32, i32, st, f32, vp, vp, ctypes.c_size_t, vp]
+    lib.kvc_decode_attention_paged_layers.restype = st
+    lib.kvc_decode_attention_paged_layers.argtypes = [
+        vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
         i32, i32, st, f32, vp, vp, ctypes.c_size_t, vp]
     lib.kvc_decode_attention_paged_noalloc.restype = st
     lib.kvc_decode_attention_paged_noalloc.argtypes = [
@@ -198,6 +203,19 @@ def kvc_decode_attention_paged(q_bf16, cache: kvc_paged_cache, block_table, olde
         hp_mode, float(softmax_scale), _ptr(out), _ptr(workspace), int(workspace_bytes),
         _stream(stream)),
         "kvc_decode_attention_paged")
+
+
+def kvc_decode_attention_paged_layers(q_bf16, cache: kvc_paged_cache, block_table, older_fmt,
+                                      context_lens, n_layers, batch, n_q_heads, n_kv_heads, head_dim,
+                                      page_size, max_pages, sink_tokens, window_tokens, hp_mode,
+                                      softmax_scale, out, workspace, workspace_bytes, stream=None) -> None:
+    """All layers of one decode step in one launch (see include/kvc.h)."""
+    _check(_lib.kvc_decode_attention_paged_layers(
+        _ptr(q_bf16), ctypes.byref(cache), _ptr(block_table), _ptr(older_fmt), _ptr(context_lens),
+        n_layers, batch, n_q_heads, n_kv_heads, head_dim, page_size, max_pages, sink_tokens,
+        window_tokens, hp_mode, float(softmax_scale), _ptr(out), _ptr(workspace), int(workspace_bytes),
+        _stream(stream)),
+        "kvc_decode_attention_paged_layers")
 
 
 def kvc_decode_read_error(workspace, batch, n_q_heads, n_kv_heads, head_dim, max_pages,

@@ -51,14 +51,20 @@ class DevicePagedCache:
     struct: K.kvc_paged_cache
     n_kv_heads: int
     head_dim: int
+    n_layers: int = 1              # pools hold n_layers * pool_pages pages, layer-major
 
     def pool_bytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in self.pools.values())
 
 
 def allocate_device_cache(layout: PagedCacheLayout, n_kv_heads: int, head_dim: int,
-                          device) -> DevicePagedCache:
-    n_bf, n_f8, n_t = layout.pool_pages
+                          device, n_layers: int = 1) -> DevicePagedCache:
+    """Pools for n_layers attention layers that share the placement: slot s
+    of layer l is pool page l * pool_pages[f] + s (the layout of
+    kvc_decode_attention_paged_layers); the struct carries the per-layer
+    counts.  page_ids address logical pages of a [n_layers * B * max_pages]
+    source, layer-major."""
+    n_bf, n_f8, n_t = (n * n_layers for n in layout.pool_pages)
     P, H, D = K.PAGE_SIZE, n_kv_heads, head_dim
     pools = {
         "k_bf16": torch.empty((n_bf, H, P, D), dtype=torch.bfloat16, device=device),
@@ -74,9 +80,11 @@ def allocate_device_cache(layout: PagedCacheLayout, n_kv_heads: int, head_dim: i
     }
     struct = K.make_paged_cache(n_pages=layout.pool_pages,
                                 **{k: (v if v.numel() else None) for k, v in pools.items()})
+    per_layer = layout.block_table.numel()
+    ids = [torch.cat([ids + l * per_layer for l in range(n_layers)]) for ids in layout.pool_src_ids]
     return DevicePagedCache(layout=layout, block_table=layout.block_table.to(device),
-                            pools=pools, page_ids=[ids.to(device) for ids in layout.pool_src_ids],
-                            struct=struct, n_kv_heads=n_kv_heads, head_dim=head_dim)
+                            pools=pools, page_ids=[i.to(device) for i in ids],
+                            struct=struct, n_kv_heads=n_kv_heads, head_dim=head_dim, n_layers=n_layers)
 
 
 def compress_into(cache: DevicePagedCache, k_pages: torch.Tensor, v_pages: torch.Tensor,
@@ -90,7 +98,7 @@ def compress_into(cache: DevicePagedCache, k_pages: torch.Tensor, v_pages: torch
             (K.KVC_FMT_BF16, ("k_bf16", "v_bf16", None, None)),
             (K.KVC_FMT_FP8_E4M3, ("k_fp8", "v_fp8", "k_fp8_scale", "v_fp8_scale")),
             (K.KVC_FMT_TERNARY2, ("k_tern", "v_tern", "k_gamma", "v_gamma"))):
-        n = cache.layout.pool_pages[fmt]
+        n = cache.layout.pool_pages[fmt] * cache.n_layers
         if n == 0:
             continue
         ids = cache.page_ids[fmt]

@@ -275,6 +275,34 @@ KVC_API kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_page
                                       size_t workspace_bytes, kvc_stream_t stream);
 
 /*
+ * kvc_decode_attention_paged_layers - the same decode attention for all
+ * attention layers of one decode step in a single launch (a step of a
+ * multi-layer model replays one launch instead of one per layer; Minima-KV,
+ * "What the memory measurements showed", runs its direct decode under CUDA
+ * graphs).  Layers share the page placement: one block table, one set of
+ * page tags and lengths; each layer has its own pools and queries.
+ *
+ *   q_bf16        device bf16 [n_layers][batch][Hq][D]
+ *   cache         pools holding n_layers * n_pages[f] pages of each format:
+ *                 slot s of layer l is page l * n_pages[f] + s (n_pages are
+ *                 the per-layer pool sizes; gamma / FP8 scales likewise)
+ *   block_table, older_fmt, context_lens   as for one layer, [batch][...]
+ *   out           device float32 [n_layers][batch][Hq][D]
+ *   workspace     >= kvc_decode_workspace_size(n_layers * batch, ...) bytes
+ * Everything else as kvc_decode_attention_paged, which is this call with
+ * n_layers = 1.  INVALID_ARG also for n_layers < 1 or n_layers * batch
+ * above 2^30.
+ */
+KVC_API kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged_cache* cache,
+                                                     const int32_t* block_table, const uint8_t* older_fmt,
+                                                     const int32_t* context_lens, int n_layers, int batch,
+                                                     int n_q_heads, int n_kv_heads, int head_dim,
+                                                     int page_size, int max_pages, int sink_tokens,
+                                                     int window_tokens, kvc_format hp_mode,
+                                                     float softmax_scale, float* out, void* workspace,
+                                                     size_t workspace_bytes, kvc_stream_t stream);
+
+/*
  * kvc_decode_read_error - synchronise `stream`, then read and clear the
  * device error flags in `workspace` (as sized for these shapes).  *flags
  * receives a bit mask: 1 = block-table entry out of range, 2 = unknown page
