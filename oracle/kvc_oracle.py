@@ -561,6 +561,77 @@ def append_retier(cache: PagedCache, block_table, context_lens, k_new, v_new, te
 
 
 # ---------------------------------------------------------------------------
+# Stale -> Anchor promotion  [Minima, "Recent, Anchor and Stale": critical
+# older pages are kept at higher fidelity as anchors, stale pages stay
+# addressable in compressed form and can be reconstructed]
+# ---------------------------------------------------------------------------
+
+PROMOTE_SLOT = 1        # flag: a ternary or anchor slot outside its pool
+PROMOTE_NOT_STALE = 2   # flag: the page is not a ternary page (sink, window or anchor)
+PROMOTE_RANGE = 4       # flag: sequence or page index outside the batch / the sequence
+
+
+def promote_pages(cache: PagedCache, block_table, older_fmt, context_lens, req_seq, req_page,
+                  anchor_slot, sink: int, window: int, hp_fmt: int, anchor_fmt: int):
+    """Re-expand selected stale (ternary) pages into anchors of format
+    ``anchor_fmt`` (BF16 or FP8), K and V alike.  Request i names logical
+    page req_page[i] of sequence req_seq[i] and the anchor-pool slot
+    anchor_slot[i] it moves to.  The page's content is its dequantised value
+    bf16(gamma * c) per KV head (the only content a stale page has); a BF16
+    anchor stores those bf16 values, an FP8 anchor quantises the bf16 page
+    with the FP8 page codec (one scale over all KV heads).  The page's
+    block-table entry becomes the anchor slot, its tag becomes anchor_fmt and
+    the ternary slot is reported as freed.
+
+    Requests that name a page outside the batch or beyond the sequence's
+    pages (PROMOTE_RANGE), a page that is not ternary by the page
+    classification (PROMOTE_NOT_STALE) or a slot outside its pool
+    (PROMOTE_SLOT) are skipped with freed = -1 and the flag OR-ed into the
+    returned word.  Requests name distinct pages.
+
+    Returns (cache', block_table', older_fmt', freed int32 [n], flags); the
+    inputs are not modified."""
+    import copy
+    c = copy.deepcopy(cache)
+    bt = np.array(block_table, dtype=np.int32, copy=True)
+    tags = np.array(older_fmt, dtype=np.uint8, copy=True)
+    n = len(req_seq)
+    freed = np.full(n, -1, dtype=np.int32)
+    flags = 0
+    n_tern = c.k_tern.shape[0]
+    n_anchor = (c.k_bf16 if anchor_fmt == BF16 else c.k_fp8).shape[0]
+    for i in range(n):
+        b, j = int(req_seq[i]), int(req_page[i])
+        if not (0 <= b < bt.shape[0]):
+            flags |= PROMOTE_RANGE
+            continue
+        L = int(context_lens[b])
+        if not (0 <= j < num_pages(L)) or L > bt.shape[1] * PAGE_SIZE:
+            flags |= PROMOTE_RANGE
+            continue
+        if page_format(j, L, sink, window, hp_fmt, int(tags[b, j])) != TERNARY:
+            flags |= PROMOTE_NOT_STALE
+            continue
+        t, a = int(bt[b, j]), int(anchor_slot[i])
+        if not (0 <= t < n_tern and 0 <= a < n_anchor):
+            flags |= PROMOTE_SLOT
+            continue
+        for which in ("k", "v"):
+            page = dequantize_ternary(getattr(c, which + "_tern")[t:t + 1],
+                                      getattr(c, which + "_gamma")[t:t + 1])        # [1][Hkv][P][D]
+            if anchor_fmt == BF16:
+                getattr(c, which + "_bf16")[a] = page[0]
+            else:
+                e, sc = quantize_fp8_pages(page)
+                getattr(c, which + "_fp8")[a] = e[0]
+                getattr(c, which + "_fp8_scale")[a] = sc[0]
+        bt[b, j] = a
+        tags[b, j] = anchor_fmt
+        freed[i] = t
+    return c, bt, tags, freed, flags
+
+
+# ---------------------------------------------------------------------------
 # Storage accounting  [Vantage, "Core architecture"; Minima, "Why the KV cache
 # becomes a bottleneck" and "What the memory measurements showed"]
 # ---------------------------------------------------------------------------

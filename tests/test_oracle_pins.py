@@ -591,3 +591,135 @@ def test_append_retier_keeps_sinks_and_anchors():
     assert freed[0] == -1 and bt_out[0, 1] == bt3[0, 1]
     out2, bt_out2, freed2, _ = O.append_retier(c3, bt3, [L3], nz, nz, [0], 4, 16, O.BF16)
     assert freed2[0] == bt3[0, 1] and bt_out2[0, 1] == 0
+
+
+# ------------------------------------------------- stale -> anchor promotion
+
+def _one_stale_page_cache(codes, gammas, n_anchor=2, d=8):
+    """A cache whose only ternary page holds the given literal packed bytes
+    ([Hkv][P][D/4]) and gammas, plus empty BF16 / FP8 anchor pools of
+    n_anchor slots; sequence 0 has 3 pages, page 1 is the stale one."""
+    hkv = codes.shape[0]
+    z16 = np.zeros((n_anchor, hkv, 16, d), np.uint16)
+    z8 = np.zeros((n_anchor, hkv, 16, d), np.uint8)
+    cache = O.PagedCache(k_bf16=z16, v_bf16=z16.copy(), k_fp8=z8, v_fp8=z8.copy(),
+                         k_fp8_scale=np.zeros(n_anchor, np.float32), v_fp8_scale=np.zeros(n_anchor, np.float32),
+                         k_tern=codes[None].copy(), v_tern=codes[None, :, ::-1].copy(),
+                         k_gamma=np.float32(gammas)[None], v_gamma=np.float32(gammas)[None].copy())
+    bt = np.array([[0, 0, 0]], np.int32)
+    tags = np.full((1, 3), O.TERNARY, np.uint8)
+    return cache, bt, tags
+
+
+def _literal_codes(hkv=4, d=8):
+    # row t of every head: bytes 0x55 (+1 +1 +1 +1), 0xFF (-1 x4), 0x1D (+1 -1 +1 0)
+    # and 0x00, rotating with t; head 3 is all zero
+    pat = [0x55, 0xFF, 0x1D, 0x00]
+    c = np.zeros((hkv, 16, d // 4), np.uint8)
+    for h in range(hkv - 1):
+        for t in range(16):
+            for w in range(d // 4):
+                c[h, t, w] = pat[(t + w + h) % 4]
+    return c
+
+
+def test_promote_bf16_literal_values():
+    # gamma 1, 0.5, 0.25 (bf16-exact) and 2.0 on an all-zero head: the anchor
+    # page holds +-gamma as bf16 bit patterns written out by hand
+    codes = _literal_codes()
+    cache, bt, tags = _one_stale_page_cache(codes, [1.0, 0.5, 0.25, 2.0])
+    out, bt2, tags2, freed, flags = O.promote_pages(cache, bt, tags, [40], [0], [1], [1], 4, 8, O.BF16, O.BF16)
+    assert flags == 0 and freed.tolist() == [0] and bt2[0, 1] == 1 and tags2[0, 1] == O.BF16
+    assert bt2[0, 0] == 0 and tags2[0, 0] == O.TERNARY and bt2[0, 2] == 0
+    pos = {0: 0x3F80, 1: 0x3F00, 2: 0x3E80, 3: 0x4000}      # 1.0, 0.5, 0.25, 2.0
+    val = {0x55: [1, 1, 1, 1], 0xFF: [-1, -1, -1, -1], 0x1D: [1, -1, 1, 0], 0x00: [0, 0, 0, 0]}
+    for h in range(4):
+        for t in range(16):
+            row = [c for w in range(2) for c in val[int(codes[h, t, w])]]
+            want = [0 if c == 0 else (pos[h] | (0x8000 if c < 0 else 0)) for c in row]
+            assert out.k_bf16[1, h, t].tolist() == want, (h, t)
+    assert np.all(out.k_bf16[0] == 0)                 # the other anchor slot untouched
+    assert np.array_equal(out.k_tern, cache.k_tern)   # the stale copy stays (freed, not erased)
+
+
+def test_promote_fp8_literal_codes_and_zero_head_excluded_from_amax():
+    # amax over the decoded page is 1.0 (the all-zero head's gamma 2.0 does not
+    # count): s = fl32(1/448); +-1, +-0.5, +-0.25 map to +-448, +-224, +-112,
+    # e4m3 0x7E, 0x76, 0x6E (sign bit 0x80), zero to 0x00
+    codes = _literal_codes()
+    cache, bt, tags = _one_stale_page_cache(codes, [1.0, 0.5, 0.25, 2.0])
+    out, bt2, tags2, freed, flags = O.promote_pages(cache, bt, tags, [40], [0], [1], [0], 4, 8, O.BF16,
+                                                    O.FP8_E4M3)
+    assert flags == 0 and freed.tolist() == [0] and bt2[0, 1] == 0 and tags2[0, 1] == O.FP8_E4M3
+    assert out.k_fp8_scale[0] == np.float32(1.0 / 448.0)
+    mag = {0: 0x7E, 1: 0x76, 2: 0x6E, 3: 0x00}
+    val = {0x55: [1, 1, 1, 1], 0xFF: [-1, -1, -1, -1], 0x1D: [1, -1, 1, 0], 0x00: [0, 0, 0, 0]}
+    for h in range(4):
+        for t in range(16):
+            row = [c for w in range(2) for c in val[int(codes[h, t, w])]]
+            want = [0 if c == 0 else (mag[h] | (0x80 if c < 0 else 0)) for c in row]
+            assert out.k_fp8[0, h, t].tolist() == want, (h, t)
+    # V was built from the row-reversed codes: same magnitudes, same scale
+    assert out.v_fp8_scale[0] == np.float32(1.0 / 448.0)
+
+
+def test_promote_skips_sinks_window_anchors_and_bad_indices():
+    codes = _literal_codes()
+    cache, bt, tags = _one_stale_page_cache(codes, [1.0, 0.5, 0.25, 2.0])
+    tags_anchor = tags.copy()
+    tags_anchor[0, 1] = O.BF16
+    cases = [
+        (dict(req_page=[0]), tags, O.PROMOTE_NOT_STALE),        # sink page
+        (dict(req_page=[2]), tags, O.PROMOTE_NOT_STALE),        # window page (L = 40, window 8)
+        (dict(req_page=[1]), tags_anchor, O.PROMOTE_NOT_STALE),  # already an anchor
+        (dict(req_page=[3]), tags, O.PROMOTE_RANGE),            # beyond the sequence's 3 pages
+        (dict(req_seq=[1]), tags, O.PROMOTE_RANGE),             # beyond the batch
+        (dict(slot=[2]), tags, O.PROMOTE_SLOT),                 # anchor pool has 2 slots
+    ]
+    for over, tg, flag in cases:
+        a = dict(req_seq=[0], req_page=[1], slot=[0])
+        a.update(over)
+        out, bt2, tags2, freed, flags = O.promote_pages(cache, bt, tg, [40], a["req_seq"], a["req_page"],
+                                                        a["slot"], 4, 8, O.BF16, O.BF16)
+        assert flags == flag and freed.tolist() == [-1], over
+        assert np.array_equal(bt2, bt) and np.array_equal(tags2, tg)
+        assert np.all(out.k_bf16 == 0) and np.all(out.v_bf16 == 0)
+
+
+@pytest.mark.parametrize("anchor_fmt", [O.BF16, O.FP8_E4M3])
+def test_promote_keeps_attention_when_values_are_exact(anchor_fmt):
+    """Groups whose |x| is one bf16 value a per (page, head) have gamma = a
+    and decode exactly to +-a; promoting such pages must leave decode
+    attention unchanged (BF16: the same values; FP8: s*e = a up to the fp32
+    rounding of s when a / amax is a power of two)."""
+    rng = np.random.default_rng(21)
+    B, maxp, hkv, d, hq = 2, 6, 2, 16, 4
+    lens = [16 * 6, 16 * 5 + 3]
+    mag = np.float32(2.0) ** rng.integers(-2, 2, size=(B, maxp, hkv))[..., None, None]
+    x = np.sign(rng.standard_normal((B, maxp, hkv, 16, d))).astype(np.float32) * mag
+    kb = bf16_bits(x)
+    vb = bf16_bits(x[:, :, ::-1])
+    q = bf16_bits(rng.standard_normal((B, hq, d)))
+    tags = np.full((B, maxp), O.TERNARY, np.uint8)
+    cache, bt, fmt = O.build_paged_cache(kb, vb, lens, 4, 20, O.BF16, older_fmt=tags)
+    ref = O.decode_attention(q, cache, bt, fmt, lens, hkv)
+    stale = [(b, j) for b in range(B) for j in range(maxp) if fmt[b, j] == O.TERNARY]
+    assert len(stale) >= 4
+    pick = stale[::2]
+    for w in ("k", "v"):                                 # room for the anchors
+        if anchor_fmt == O.BF16:
+            setattr(cache, w + "_bf16", np.concatenate([getattr(cache, w + "_bf16"),
+                                                        np.zeros((len(pick), hkv, 16, d), np.uint16)]))
+        else:
+            setattr(cache, w + "_fp8", np.zeros((len(pick), hkv, 16, d), np.uint8))
+            setattr(cache, w + "_fp8_scale", np.zeros(len(pick), np.float32))
+    base = 0 if anchor_fmt == O.FP8_E4M3 else cache.k_bf16.shape[0] - len(pick)
+    slots = [base + i for i in range(len(pick))]
+    out, bt2, tags2, freed, flags = O.promote_pages(cache, bt, tags, lens, [b for b, _ in pick],
+                                                    [j for _, j in pick], slots, 4, 20, O.BF16, anchor_fmt)
+    assert flags == 0 and sorted(freed.tolist()) == sorted(int(bt[b, j]) for b, j in pick)
+    fmt2 = np.array([[O.page_format(j, lens[b], 4, 20, O.BF16, int(tags2[b, j])) if j < O.num_pages(lens[b])
+                      else 255 for j in range(maxp)] for b in range(B)], np.uint8)
+    assert all(fmt2[b, j] == anchor_fmt for b, j in pick)
+    got = O.decode_attention(q, out, bt2, fmt2, lens, hkv)
+    assert np.abs(got - ref).max() < (1e-12 if anchor_fmt == O.BF16 else 1e-6)
