@@ -149,16 +149,20 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
+def ncu_traffic(kernel_key, workload):
     """dram bytes per launch recorded from an ncu capture of the current
-    kernel sources (profiles/ncu_traffic.txt), else None."""
+    kernel sources for this workload at its default size
+    (profiles/ncu_traffic.txt), else None."""
+    if workload is None:
+        return None
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
     src = kernel_source_hash()
     for line in open(path):
         parts = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
-        if parts.get("kernel") == kernel_key and parts.get("sources") == src and "bytes_per_launch" in parts:
+        if (parts.get("kernel") == kernel_key and parts.get("sources") == src and
+                parts.get("workload") == workload and "bytes_per_launch" in parts):
             return float(parts["bytes_per_launch"])
     return None
 
@@ -305,7 +309,7 @@ def run_ours(args, rank, world, dev, peak, peak_src):
 
     def roof(name):
         k = kernels[name]
-        traffic = ncu_traffic(name)
+        traffic = ncu_traffic(name, args.workload if args.batch is None and args.layers is None else None)
         return {"bound": "hbm", "achieved": k["gbs"], "peak": peak, "unit": "GB/s",
                 "frac": k["frac"], "traffic": traffic, "kernel": name, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": k["bytes"]}
@@ -321,6 +325,10 @@ def run_ours(args, rank, world, dev, peak, peak_src):
                                                        hp, peak)
     if ap is not None:
         res["kernels"]["append_retier"] = ap
+    pr = None if n_layers > 1 else time_promote(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp,
+                                                 peak)
+    if pr is not None:
+        res["kernels"]["promote"] = pr
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out,
                              step_bytes, world, dev, hp, n_layers)
@@ -399,6 +407,105 @@ def time_append_retier(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp,
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes": int(nbytes),
             "share": None, "sequences_retiered": n_ret, "note": "one decode step's append + retier, not in the step"}
+
+
+def time_promote(args, K, cfg, cache, lens, older, B, H, D, max_pages, hp, peak, per_seq=32):
+    """The stale-to-anchor row of the design: kvc_promote_pages re-expands
+    per_seq stale pages of every sequence (spread over its stale range) into
+    anchors of the high-precision format, timed alone and not part of the
+    step.  The anchors go to scratch pools (the struct's anchor pools are
+    replaced by them); a scratch block table and tag array are restored
+    before each call."""
+    dev = lens.device
+    L = lens.cpu().tolist()
+    tags_h = None if older is None else older.cpu()
+    reqs = []
+    for b in range(B):
+        first = -(-cfg["sink"] // P)                            # first page past the sinks
+        last = max(0, (L[b] - cfg["window"]) // P)              # pages before the window's first
+        cand = [j for j in range(first, last) if tags_h is None or int(tags_h[b, j]) == K.KVC_FMT_TERNARY2]
+        if len(cand) >= per_seq:
+            step = len(cand) // per_seq
+            reqs += [(b, cand[i * step]) for i in range(per_seq)]
+    if not reqs:
+        return None
+    n = len(reqs)
+    bf = hp == K.KVC_FMT_BF16
+    ak = torch.empty((n, H, P, D), dtype=torch.bfloat16 if bf else torch.uint8, device=dev)
+    av = torch.empty_like(ak)
+    sk = torch.empty(n, dtype=torch.float32, device=dev)
+    sv = torch.empty_like(sk)
+    st = K.kvc_paged_cache()
+    ctypes_copy(st, cache.struct)
+    if bf:
+        st.k_bf16, st.v_bf16 = ak.data_ptr(), av.data_ptr()
+    else:
+        st.k_fp8, st.v_fp8 = ak.data_ptr(), av.data_ptr()
+        st.k_fp8_scale, st.v_fp8_scale = sk.data_ptr(), sv.data_ptr()
+    st.n_pages[hp] = n
+    bt0 = cache.block_table.clone()
+    bt = bt0.clone()
+    tags0 = (torch.full((B, max_pages), K.KVC_FMT_TERNARY2, dtype=torch.uint8, device=dev) if older is None
+             else older.clone())
+    tags = tags0.clone()
+    seq = torch.tensor([r[0] for r in reqs], dtype=torch.int32, device=dev)
+    page = torch.tensor([r[1] for r in reqs], dtype=torch.int32, device=dev)
+    slot = torch.arange(n, dtype=torch.int32, device=dev)
+    freed = torch.empty(n, dtype=torch.int32, device=dev)
+    flags = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def restore():
+        bt.copy_(bt0)
+        tags.copy_(tags0)
+
+    def one():
+        restore()
+        K.kvc_promote_pages(st, bt, tags, lens, seq, page, slot, n, freed, flags, B, H, D, P, max_pages,
+                            cfg["sink"], cfg["window"], hp, hp)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    if int(flags.item()) or int((freed < 0).sum().item()):
+        raise RuntimeError(f"promote device flags {int(flags.item())}")
+    reps = 20
+    g_full, g_copy = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_full):
+        for _ in range(reps):
+            one()
+    with torch.cuda.graph(g_copy):
+        for _ in range(reps):
+            restore()
+    times = []
+    for g in (g_full, g_copy):
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / (5 * reps))
+    del g_full, g_copy
+    ms = max(times[0] - times[1], 1e-6)
+    per_page = 2 * H * (P * D // 4 + 4) + 2 * H * P * D * (2 if bf else 1) + (0 if bf else 8)
+    nbytes = n * per_page
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes": int(nbytes),
+            "share": None, "pages_promoted": n,
+            "note": f"{n} stale pages re-expanded to {'BF16' if bf else 'FP8'} anchors, not in the step"}
+
+
+def ctypes_copy(dst, src):
+    for name, _ in src._fields_:
+        if name == "n_pages":
+            for f in range(3):
+                dst.n_pages[f] = src.n_pages[f]
+        else:
+            setattr(dst, name, getattr(src, name))
 
 
 def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, out, step_bytes,
@@ -557,7 +664,7 @@ def run_bulk(args, rank, world, dev, peak, peak_src):
     def roof(name):
         k = kernels[name]
         return {"bound": "hbm", "achieved": k["gbs"], "peak": peak, "unit": "GB/s", "frac": k["frac"],
-                "traffic": ncu_traffic(name), "kernel": name, "peak_source": peak_src,
+                "traffic": ncu_traffic(name, "bulk"), "kernel": name, "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": k["bytes"]}
 
     res = {"value": step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9,

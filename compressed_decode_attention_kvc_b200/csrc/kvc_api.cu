@@ -161,6 +161,40 @@ kvc_status kvc_append_retier(const void* k_new_bf16, const void* v_new_bf16,
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+kvc_status kvc_promote_pages(const kvc_paged_cache* cache, int32_t* block_table, uint8_t* older_fmt,
+                             const int32_t* context_lens, const int32_t* req_seq, const int32_t* req_page,
+                             const int32_t* anchor_slot, int n_requests, int32_t* freed_ternary_slot,
+                             uint32_t* device_flags, int batch, int n_kv_heads, int head_dim, int page_size,
+                             int max_pages, int sink_tokens, int window_tokens, kvc_format hp_mode,
+                             kvc_format anchor_fmt, kvc_stream_t stream) {
+  if (n_requests < 0 || batch < 0 || n_kv_heads < 1 || max_pages < 1 || sink_tokens < 0 || window_tokens < 0)
+    return KVC_ERR_INVALID_ARG;
+  if (page_size != KVC_PAGE_SIZE || !head_dim_ok(head_dim)) return KVC_ERR_UNSUPPORTED;
+  if (hp_mode != KVC_FMT_BF16 && hp_mode != KVC_FMT_FP8_E4M3) return KVC_ERR_INVALID_ARG;
+  if (anchor_fmt != KVC_FMT_BF16 && anchor_fmt != KVC_FMT_FP8_E4M3) return KVC_ERR_INVALID_ARG;
+  if (!cache) return KVC_ERR_INVALID_ARG;
+  if (n_requests == 0) return KVC_OK;
+  if ((long long)batch * max_pages > 0x7fffffffll) return KVC_ERR_UNSUPPORTED;
+  if (!block_table || !older_fmt || !context_lens || !req_seq || !req_page || !anchor_slot ||
+      !freed_ternary_slot)
+    return KVC_ERR_INVALID_ARG;
+  const bool bf = anchor_fmt == KVC_FMT_BF16;
+  const void* ak = bf ? cache->k_bf16 : cache->k_fp8;
+  const void* av = bf ? cache->v_bf16 : cache->v_fp8;
+  if (cache->n_pages[anchor_fmt] > 0 && (!ak || !av || !aligned(ak, 16) || !aligned(av, 16)))
+    return KVC_ERR_INVALID_ARG;
+  if (!bf && cache->n_pages[anchor_fmt] > 0 && (!cache->k_fp8_scale || !cache->v_fp8_scale))
+    return KVC_ERR_INVALID_ARG;
+  if (cache->n_pages[KVC_FMT_TERNARY2] > 0 &&
+      (!cache->k_tern || !cache->v_tern || !cache->k_gamma || !cache->v_gamma ||
+       !aligned(cache->k_tern, 16) || !aligned(cache->v_tern, 16)))
+    return KVC_ERR_INVALID_ARG;
+  return from_cuda(kvc::launch_promote(*cache, block_table, older_fmt, context_lens, req_seq, req_page,
+                                       anchor_slot, freed_ternary_slot, device_flags, n_requests, batch,
+                                       n_kv_heads, head_dim, max_pages, sink_tokens, window_tokens, hp_mode,
+                                       anchor_fmt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvc_status kvc_plan_paged_cache(const int32_t* context_lens, int batch, int max_pages,
                                 int page_size, int sink_tokens, int window_tokens,
                                 kvc_format hp_mode, const uint8_t* older_fmt,

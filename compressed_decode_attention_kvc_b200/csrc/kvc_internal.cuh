@@ -42,6 +42,11 @@ cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const in
 cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids,
                                int n, int hkv, int d, void* dst, cudaStream_t s);
 
+cudaError_t launch_promote(const kvc_paged_cache& cache, int32_t* block_table, uint8_t* older_fmt,
+                           const int32_t* ctx, const int32_t* req_seq, const int32_t* req_page,
+                           const int32_t* anchor_slot, int32_t* freed, uint32_t* flags, int n, int batch,
+                           int hkv, int d, int max_pages, int sink, int window, int hp, int anchor,
+                           cudaStream_t s);
 cudaError_t launch_append_retier(const void* k_new, const void* v_new, const kvc_paged_cache& cache,
                                 int32_t* block_table, uint8_t* older_fmt, const int32_t* ctx,
                                 const int32_t* tern_slot, int32_t* freed, uint32_t* flags, int batch,

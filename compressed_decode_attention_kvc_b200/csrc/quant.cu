@@ -454,6 +454,147 @@ __global__ void __launch_bounds__(256) append_retier_kernel(AppendParams p) {
   }
 }
 
+// ------------------------------------------------ stale -> anchor promotion
+// Minima-KV, "Recent, Anchor and Stale": critical older pages are kept at
+// higher fidelity as anchors while stale pages stay addressable in
+// compressed form.  One CTA per request re-expands a stale (ternary) page
+// into an anchor slot of the BF16 or FP8 pools: the page's content is
+// bf16(gamma * c) per KV head; an FP8 anchor encodes that bf16 page with the
+// FP8 page codec (one scale over all KV heads, K and V separately).  The
+// block-table entry moves to the anchor slot, the tag becomes the anchor
+// format, and the ternary slot is reported as freed.
+struct PromoteParams {
+  kvc_paged_cache cache;
+  int32_t* block_table;       // [batch][max_pages]
+  uint8_t* older_fmt;         // [batch][max_pages]
+  const int32_t* ctx;         // [batch]
+  const int32_t* req_seq;     // [n]
+  const int32_t* req_page;    // [n]
+  const int32_t* anchor_slot; // [n]
+  int32_t* freed;             // [n] out
+  uint32_t* flags;            // device error word or null
+  int batch, Hkv, max_pages, sink, window, hp, anchor;
+};
+
+// bf16 bit patterns of the 8 codes of one 16-bit word (2 bits each, LSB
+// first): +1 -> pos, -1 -> neg, 0 and the unused field 10 -> +0.
+__device__ __forceinline__ uint4 tern8_to_bf16(uint32_t w, uint32_t pos, uint32_t neg) {
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t f0 = (w >> (4 * k)) & 3u, f1 = (w >> (4 * k + 2)) & 3u;
+    const uint32_t lo = f0 == 1u ? pos : (f0 == 3u ? neg : 0u);
+    const uint32_t hi = f1 == 1u ? pos : (f1 == 3u ? neg : 0u);
+    o[k] = lo | (hi << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) promote_kernel(PromoteParams p) {
+  constexpr int NC = D / 16;                 // 16-bit code words per lane per group
+  __shared__ uint32_t amax_bits[2];          // K, V: amax of the decoded page (float bits, >= 0)
+  const int i = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = p.req_seq[i], j = p.req_page[i];
+  uint32_t flag = 0;
+  long long row = 0;
+  int t = -1, a = -1;
+  if (b < 0 || b >= p.batch) {
+    flag = kErrContext;
+  } else {
+    const int L = p.ctx[b];
+    if (L < 0 || L > p.max_pages * kPage || j < 0 || j >= (L + kPage - 1) / kPage) {
+      flag = kErrContext;
+    } else {
+      row = (long long)b * p.max_pages + j;
+      if (page_format(j, L, p.sink, p.window, p.hp, p.older_fmt[row]) != KVC_FMT_TERNARY2) {
+        flag = kErrFormat;
+      } else {
+        t = p.block_table[row];
+        a = p.anchor_slot[i];
+        const long long n_anchor = p.anchor == KVC_FMT_BF16 ? p.cache.n_pages[0] : p.cache.n_pages[1];
+        if (t < 0 || t >= p.cache.n_pages[2] || a < 0 || a >= n_anchor) flag = kErrBlockTable;
+      }
+    }
+  }
+  if (flag) {                                // uniform across the CTA
+    if (threadIdx.x == 0) {
+      if (p.flags) atomicOr(p.flags, flag);
+      p.freed[i] = -1;
+    }
+    return;
+  }
+  const int n_groups = 2 * p.Hkv;            // K heads, then V heads
+  const bool fp8 = p.anchor == KVC_FMT_FP8_E4M3;
+  if (fp8) {
+    if (threadIdx.x < 2) amax_bits[threadIdx.x] = 0u;
+    __syncthreads();
+    // amax of the decoded page: bf16(gamma) of every head with a nonzero code
+    for (int g = warp; g < n_groups; g += 8) {
+      const bool is_v = g >= p.Hkv;
+      const int h = is_v ? g - p.Hkv : g;
+      const long long grp = (long long)t * p.Hkv + h;
+      const uint16_t* src = static_cast<const uint16_t*>(is_v ? p.cache.v_tern : p.cache.k_tern) + grp * (2 * D);
+      uint32_t any = 0;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) any |= src[c * 32 + lane];
+      if (__any_sync(0xffffffffu, (any & 0x5555u) != 0u) && lane == 0) {
+        const float gam = (is_v ? p.cache.v_gamma : p.cache.k_gamma)[grp];
+        const float x = __bfloat162float(__float2bfloat16_rn(gam));
+        atomicMax(&amax_bits[is_v ? 1 : 0], __float_as_uint(fabsf(x)));
+      }
+    }
+    __syncthreads();
+  }
+  for (int g = warp; g < n_groups; g += 8) {
+    const bool is_v = g >= p.Hkv;
+    const int h = is_v ? g - p.Hkv : g;
+    const long long grp = (long long)t * p.Hkv + h, dgrp = (long long)a * p.Hkv + h;
+    const uint16_t* src = static_cast<const uint16_t*>(is_v ? p.cache.v_tern : p.cache.k_tern) + grp * (2 * D);
+    const float gam = (is_v ? p.cache.v_gamma : p.cache.k_gamma)[grp];
+    const uint32_t pos = __bfloat16_as_ushort(__float2bfloat16_rn(gam));
+    const uint32_t neg = pos ^ 0x8000u;
+    uint32_t w[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) w[c] = src[c * 32 + lane];
+    if (!fp8) {
+      uint4* dst = static_cast<uint4*>(const_cast<void*>(is_v ? p.cache.v_bf16 : p.cache.k_bf16)) + dgrp * (2 * D);
+#pragma unroll
+      for (int c = 0; c < NC; ++c) dst[c * 32 + lane] = tern8_to_bf16(w[c], pos, neg);
+    } else {
+      // the FP8 page codec on the decoded values: y = fl32(x * fl32(448 / amax)),
+      // RNE-satfinite e4m3; a head takes only the values +-bf16(gamma) and +0
+      const float amax = __uint_as_float(amax_bits[is_v ? 1 : 0]);
+      const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
+      const float x = __uint_as_float(pos << 16);
+      const float2 y = make_float2(__fmul_rn(x, inv), __fmul_rn(-x, inv));
+      const uint32_t e2 = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+      const uint32_t ep = e2 & 0xFFu, en = (e2 >> 8) & 0xFFu;
+      uint2* dst = static_cast<uint2*>(const_cast<void*>(is_v ? p.cache.v_fp8 : p.cache.k_fp8)) + dgrp * (2 * D);
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        uint32_t o[2] = {0u, 0u};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t f = (w[c] >> (2 * k)) & 3u;
+          o[k >> 2] |= (f == 1u ? ep : (f == 3u ? en : 0u)) << (8 * (k & 3));
+        }
+        dst[c * 32 + lane] = make_uint2(o[0], o[1]);
+      }
+      if (h == 0 && lane == 0)
+        const_cast<float*>(is_v ? p.cache.v_fp8_scale : p.cache.k_fp8_scale)[a] =
+            amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    }
+  }
+  __syncthreads();                           // every thread has read the entry before it changes
+  if (threadIdx.x == 0) {
+    p.block_table[row] = a;
+    p.older_fmt[row] = (uint8_t)p.anchor;
+    p.freed[i] = t;
+  }
+}
+
 int grid_for(long long work, int per_block) {
   long long g = (work + per_block - 1) / per_block;
   if (g > (1ll << 30)) g = 1ll << 30;
@@ -533,6 +674,37 @@ cudaError_t launch_append_retier(const void* k_new, const void* v_new, const kvc
     case 64: append_retier_kernel<64><<<batch, 256, 0, s>>>(p); break;
     case 128: append_retier_kernel<128><<<batch, 256, 0, s>>>(p); break;
     case 256: append_retier_kernel<256><<<batch, 256, 0, s>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_promote(const kvc_paged_cache& cache, int32_t* block_table, uint8_t* older_fmt,
+                           const int32_t* ctx, const int32_t* req_seq, const int32_t* req_page,
+                           const int32_t* anchor_slot, int32_t* freed, uint32_t* flags, int n, int batch,
+                           int hkv, int d, int max_pages, int sink, int window, int hp, int anchor,
+                           cudaStream_t s) {
+  PromoteParams p;
+  p.cache = cache;
+  p.block_table = block_table;
+  p.older_fmt = older_fmt;
+  p.ctx = ctx;
+  p.req_seq = req_seq;
+  p.req_page = req_page;
+  p.anchor_slot = anchor_slot;
+  p.freed = freed;
+  p.flags = flags;
+  p.batch = batch;
+  p.Hkv = hkv;
+  p.max_pages = max_pages;
+  p.sink = sink;
+  p.window = window;
+  p.hp = hp;
+  p.anchor = anchor;
+  switch (d) {
+    case 64: promote_kernel<64><<<n, 256, 0, s>>>(p); break;
+    case 128: promote_kernel<128><<<n, 256, 0, s>>>(p); break;
+    case 256: promote_kernel<256><<<n, 256, 0, s>>>(p); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -42,7 +42,7 @@ EXPORTS = (
     "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
     "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc", "kvc_append_retier",
-    "kvc_decode_attention_paged_layers",
+    "kvc_decode_attention_paged_layers", "kvc_promote_pages",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -81,6 +81,9 @@ def _load() -> ctypes.CDLL:
     lib.kvc_append_retier.restype = st
     lib.kvc_append_retier.argtypes = [vp, vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, vp, vp, vp,
                                       i32, i32, i32, i32, i32, i32, i32, st, vp]
+    lib.kvc_promote_pages.restype = st
+    lib.kvc_promote_pages.argtypes = [ctypes.POINTER(kvc_paged_cache), vp, vp, vp, vp, vp, vp, i32, vp, vp,
+                                      i32, i32, i32, i32, i32, i32, i32, st, st, vp]
     lib.kvc_plan_paged_cache.restype = st
     lib.kvc_plan_paged_cache.argtypes = [vp, i32, i32, i32, i32, i32, st, vp, vp, vp, vp, vp, vp]
     lib.kvc_decode_workspace_size.restype = st
@@ -158,6 +161,19 @@ def kvc_append_retier(k_new_bf16, v_new_bf16, cache: kvc_paged_cache, block_tabl
                                   n_kv_heads, head_dim, page_size, max_pages, sink_tokens,
                                   window_tokens, hp_mode, _stream(stream)),
            "kvc_append_retier")
+
+
+def kvc_promote_pages(cache: kvc_paged_cache, block_table, older_fmt, context_lens, req_seq, req_page,
+                      anchor_slot, n_requests, freed_ternary_slot, device_flags, batch, n_kv_heads,
+                      head_dim, page_size, max_pages, sink_tokens, window_tokens, hp_mode, anchor_fmt,
+                      stream=None) -> None:
+    """Re-expand stale (ternary) pages into BF16 / FP8 anchors (see include/kvc.h)."""
+    _check(_lib.kvc_promote_pages(ctypes.byref(cache), _ptr(block_table), _ptr(older_fmt),
+                                  _ptr(context_lens), _ptr(req_seq), _ptr(req_page), _ptr(anchor_slot),
+                                  n_requests, _ptr(freed_ternary_slot), _ptr(device_flags), batch,
+                                  n_kv_heads, head_dim, page_size, max_pages, sink_tokens, window_tokens,
+                                  hp_mode, anchor_fmt, _stream(stream)),
+           "kvc_promote_pages")
 
 
 def kvc_plan_paged_cache(context_lens, batch, max_pages, page_size, sink_tokens, window_tokens,

@@ -197,6 +197,53 @@ KVC_API kvc_status kvc_append_retier(const void* k_new_bf16, const void* v_new_b
                                      int window_tokens, kvc_format hp_mode, kvc_stream_t stream);
 
 /*
+ * kvc_promote_pages - stale-to-anchor promotion: re-expand selected stale
+ * (ternary) pages into anchors, the higher-fidelity tier that Minima-KV
+ * keeps for critical older pages while stale pages stay addressable in
+ * compressed form ("Minima-KV", section "Recent, Anchor and Stale").
+ * Request i moves logical page req_page[i] of sequence req_seq[i] to slot
+ * anchor_slot[i] of the anchor_fmt pools, K and V alike.  The page's
+ * content is bf16(gamma * c) per KV head (what kvc_dequantize_pages gives);
+ * a BF16 anchor stores it as it is, an FP8 anchor encodes the bf16 page
+ * with the FP8 page codec of kvc_quantize_pack_pages (one scale over all KV
+ * heads, K and V separately; heads whose codes are all 0 add nothing to
+ * amax).  block_table[b][j] becomes the anchor slot, older_fmt[b][j]
+ * becomes anchor_fmt and freed_ternary_slot[i] the released ternary slot
+ * (the ternary bytes are left as they are).
+ *
+ *   cache          host pointer to the pools; the anchor_fmt pools (and
+ *                  their FP8 scales) are WRITTEN (pointers cast from const)
+ *   block_table    device int32 [batch][max_pages], read and updated
+ *   older_fmt      device uint8 [batch][max_pages], read and updated
+ *                  (required: the tag is what makes the page an anchor)
+ *   context_lens   device int32 [batch]
+ *   req_seq, req_page, anchor_slot  device int32 [n_requests]; requests
+ *                  name distinct pages and distinct anchor slots
+ *   freed_ternary_slot  device int32 [n_requests], out: the ternary slot,
+ *                  or -1 for a skipped request
+ *   device_flags   device uint32 word or NULL: OR-ed with 4 (sequence or
+ *                  page outside the batch / the sequence's pages), 2 (the
+ *                  page is not ternary: a sink, window or anchor page), 1
+ *                  (a ternary or anchor slot outside its pool); such a
+ *                  request is skipped and changes nothing
+ *   hp_mode        format of sink and window pages (BF16 or FP8_E4M3), for
+ *                  the page classification
+ *   anchor_fmt     BF16 or FP8_E4M3
+ * Errors: INVALID_ARG for null or misaligned pointers, negative sizes, a bad
+ * hp_mode or anchor_fmt; UNSUPPORTED for page_size != 16, a head_dim other
+ * than 64, 128, 256, or batch * max_pages >= 2^31.  Asynchronous on
+ * `stream`; allocates nothing; one CTA per request.
+ */
+KVC_API kvc_status kvc_promote_pages(const kvc_paged_cache* cache, int32_t* block_table,
+                                     uint8_t* older_fmt, const int32_t* context_lens,
+                                     const int32_t* req_seq, const int32_t* req_page,
+                                     const int32_t* anchor_slot, int n_requests,
+                                     int32_t* freed_ternary_slot, uint32_t* device_flags, int batch,
+                                     int n_kv_heads, int head_dim, int page_size, int max_pages,
+                                     int sink_tokens, int window_tokens, kvc_format hp_mode,
+                                     kvc_format anchor_fmt, kvc_stream_t stream);
+
+/*
  * kvc_plan_paged_cache - host-side page placement (a small block manager).
  * Decides each logical page's format with the same rule the decode kernel
  * applies, and gives every page a slot in the pool of its format.

@@ -150,3 +150,28 @@ def test_append_retier_argument_errors():
     assert call(ptr=0) == K.KVC_ERR_INVALID_ARG
     assert call(ptr=(1 << 20) + 8) == K.KVC_ERR_INVALID_ARG  # misaligned new-token rows
     assert call() == K.KVC_ERR_INVALID_ARG                  # no BF16 pools in the cache
+
+
+def test_promote_argument_errors():
+    """Host-side validation of kvc_promote_pages (no GPU work is launched)."""
+    import ctypes
+    lib = ctypes.CDLL(K.LIB_PATH)
+    lib.kvc_promote_pages.restype = ctypes.c_int
+    cache = K.kvc_paged_cache()
+    vp = ctypes.c_void_p
+    def call(n=1, batch=1, hkv=2, d=128, page=16, max_pages=4, sink=4, window=16, hp=K.KVC_FMT_BF16,
+             anchor=K.KVC_FMT_BF16, ptr=1 << 20, tags=True, cache_p=True):
+        p = vp(ptr) if ptr else None
+        return lib.kvc_promote_pages(ctypes.byref(cache) if cache_p else None, p, p if tags else None, p, p, p,
+                                     p, n, p, None, batch, hkv, d, page, max_pages, sink, window, hp, anchor,
+                                     None)
+    assert call(page=8) == K.KVC_ERR_UNSUPPORTED
+    assert call(d=96) == K.KVC_ERR_UNSUPPORTED
+    assert call(hp=K.KVC_FMT_TERNARY2) == K.KVC_ERR_INVALID_ARG
+    assert call(anchor=K.KVC_FMT_TERNARY2) == K.KVC_ERR_INVALID_ARG
+    assert call(n=-1) == K.KVC_ERR_INVALID_ARG
+    assert call(cache_p=False) == K.KVC_ERR_INVALID_ARG
+    assert call(n=0) == K.KVC_OK                            # nothing to do, nothing launched
+    assert call(tags=False) == K.KVC_ERR_INVALID_ARG        # the tag makes a page an anchor
+    assert call(ptr=0) == K.KVC_ERR_INVALID_ARG
+    assert call(batch=1 << 20, max_pages=1 << 12) == K.KVC_ERR_UNSUPPORTED
