@@ -195,6 +195,53 @@ kvc_status kvc_promote_pages(const kvc_paged_cache* cache, int32_t* block_table,
                                        anchor_fmt, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// values of one page of one pool, or -1 when outside the codec's range
+static long long exans_group_elems(int page_size, int n_kv_heads, int head_dim) {
+  if (page_size != KVC_PAGE_SIZE || !head_dim_ok(head_dim) || n_kv_heads < 1) return -1;
+  const long long n = (long long)n_kv_heads * KVC_PAGE_SIZE * head_dim;
+  return n <= (1ll << 22) ? n : -1;
+}
+
+kvc_status kvc_exans_workspace_size(int n, int page_size, int n_kv_heads, int head_dim, size_t* bytes) {
+  if (!bytes || n < 0) return KVC_ERR_INVALID_ARG;
+  const long long N = exans_group_elems(page_size, n_kv_heads, head_dim);
+  if (N < 0) return KVC_ERR_UNSUPPORTED;
+  *bytes = (size_t)n * (size_t)kvc::exans_slot_bytes(N);
+  return KVC_OK;
+}
+
+kvc_status kvc_exans_encode(const void* src_bf16, const int32_t* page_ids, int n, int page_size,
+                            int n_kv_heads, int head_dim, void* workspace, size_t workspace_bytes, void* dst,
+                            size_t dst_bytes, int64_t* offsets, kvc_stream_t stream) {
+  if (n < 0 || n > (1 << 24)) return KVC_ERR_INVALID_ARG;
+  const long long N = exans_group_elems(page_size, n_kv_heads, head_dim);
+  if (N < 0) return KVC_ERR_UNSUPPORTED;
+  if (!offsets) return KVC_ERR_INVALID_ARG;
+  if (n == 0) return from_cuda(cudaMemsetAsync(offsets, 0, sizeof(int64_t), reinterpret_cast<cudaStream_t>(stream)));
+  if (!src_bf16 || !dst || !aligned(src_bf16, 16) || !aligned(dst, 16) || !aligned(offsets, 8))
+    return KVC_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < (size_t)n * (size_t)kvc::exans_slot_bytes(N))
+    return KVC_ERR_WORKSPACE;
+  if (dst_bytes < (size_t)n * (size_t)(64 + 2 * N)) return KVC_ERR_INVALID_ARG;
+  return from_cuda(kvc::launch_exans_encode(src_bf16, page_ids, n, N, workspace,
+                                            reinterpret_cast<long long*>(offsets), dst,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kvc_status kvc_exans_decode(const void* src, size_t src_bytes, const int64_t* offsets, int n_blobs,
+                            const int32_t* blob_ids, int n, int page_size, int n_kv_heads, int head_dim,
+                            void* dst_bf16, uint32_t* device_flags, kvc_stream_t stream) {
+  if (n < 0 || n_blobs < 0) return KVC_ERR_INVALID_ARG;
+  const long long N = exans_group_elems(page_size, n_kv_heads, head_dim);
+  if (N < 0) return KVC_ERR_UNSUPPORTED;
+  if (n == 0) return KVC_OK;
+  if (!src || !offsets || !dst_bf16 || !aligned(src, 16) || !aligned(dst_bf16, 16) || !aligned(offsets, 8))
+    return KVC_ERR_INVALID_ARG;
+  return from_cuda(kvc::launch_exans_decode(src, (long long)src_bytes, reinterpret_cast<const long long*>(offsets),
+                                            n_blobs, blob_ids, n, N, dst_bf16, device_flags,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kvc_status kvc_plan_paged_cache(const int32_t* context_lens, int batch, int max_pages,
                                 int page_size, int sink_tokens, int window_tokens,
                                 kvc_format hp_mode, const uint8_t* older_fmt,

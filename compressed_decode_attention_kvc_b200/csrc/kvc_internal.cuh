@@ -42,6 +42,13 @@ cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const in
 cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids,
                                int n, int hkv, int d, void* dst, cudaStream_t s);
 
+// exponent-split lossless codec of BF16 pages (exans.cu)
+long long exans_slot_bytes(long long group_elems);
+cudaError_t launch_exans_encode(const void* src, const int32_t* page_ids, int n, long long group_elems,
+                                void* ws, long long* offsets, void* dst, cudaStream_t s);
+cudaError_t launch_exans_decode(const void* src, long long src_bytes, const long long* offsets, int n_blobs,
+                                const int32_t* ids, int n, long long group_elems, void* dst, uint32_t* flags,
+                                cudaStream_t s);
 cudaError_t launch_promote(const kvc_paged_cache& cache, int32_t* block_table, uint8_t* older_fmt,
                            const int32_t* ctx, const int32_t* req_seq, const int32_t* req_page,
                            const int32_t* anchor_slot, int32_t* freed, uint32_t* flags, int n, int batch,

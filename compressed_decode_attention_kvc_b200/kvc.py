@@ -42,7 +42,8 @@ EXPORTS = (
     "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
     "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc", "kvc_append_retier",
-    "kvc_decode_attention_paged_layers", "kvc_promote_pages",
+    "kvc_decode_attention_paged_layers", "kvc_promote_pages", "kvc_exans_workspace_size",
+    "kvc_exans_encode", "kvc_exans_decode",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -84,6 +85,13 @@ def _load() -> ctypes.CDLL:
     lib.kvc_promote_pages.restype = st
     lib.kvc_promote_pages.argtypes = [ctypes.POINTER(kvc_paged_cache), vp, vp, vp, vp, vp, vp, i32, vp, vp,
                                       i32, i32, i32, i32, i32, i32, i32, st, st, vp]
+    lib.kvc_exans_workspace_size.restype = st
+    lib.kvc_exans_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kvc_exans_encode.restype = st
+    lib.kvc_exans_encode.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp,
+                                     vp]
+    lib.kvc_exans_decode.restype = st
+    lib.kvc_exans_decode.argtypes = [vp, ctypes.c_size_t, vp, i32, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.kvc_plan_paged_cache.restype = st
     lib.kvc_plan_paged_cache.argtypes = [vp, i32, i32, i32, i32, i32, st, vp, vp, vp, vp, vp, vp]
     lib.kvc_decode_workspace_size.restype = st
@@ -174,6 +182,29 @@ def kvc_promote_pages(cache: kvc_paged_cache, block_table, older_fmt, context_le
                                   n_kv_heads, head_dim, page_size, max_pages, sink_tokens, window_tokens,
                                   hp_mode, anchor_fmt, _stream(stream)),
            "kvc_promote_pages")
+
+
+def kvc_exans_workspace_size(n, page_size, n_kv_heads, head_dim) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.kvc_exans_workspace_size(n, page_size, n_kv_heads, head_dim, ctypes.byref(out)),
+           "kvc_exans_workspace_size")
+    return out.value
+
+
+def kvc_exans_encode(src_bf16, page_ids, n, page_size, n_kv_heads, head_dim, workspace, workspace_bytes, dst,
+                     dst_bytes, offsets, stream=None) -> None:
+    """Lossless exponent-split coding of n BF16 pages (see include/kvc.h)."""
+    _check(_lib.kvc_exans_encode(_ptr(src_bf16), _ptr(page_ids), n, page_size, n_kv_heads, head_dim,
+                                 _ptr(workspace), int(workspace_bytes), _ptr(dst), int(dst_bytes), _ptr(offsets),
+                                 _stream(stream)),
+           "kvc_exans_encode")
+
+
+def kvc_exans_decode(src, src_bytes, offsets, n_blobs, blob_ids, n, page_size, n_kv_heads, head_dim, dst_bf16,
+                     device_flags, stream=None) -> None:
+    _check(_lib.kvc_exans_decode(_ptr(src), int(src_bytes), _ptr(offsets), n_blobs, _ptr(blob_ids), n, page_size,
+                                 n_kv_heads, head_dim, _ptr(dst_bf16), _ptr(device_flags), _stream(stream)),
+           "kvc_exans_decode")
 
 
 def kvc_plan_paged_cache(context_lens, batch, max_pages, page_size, sink_tokens, window_tokens,

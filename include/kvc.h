@@ -234,6 +234,71 @@ KVC_API kvc_status kvc_append_retier(const void* k_new_bf16, const void* v_new_b
  * than 64, 128, 256, or batch * max_pages >= 2^31.  Asynchronous on
  * `stream`; allocates nothing; one CTA per request.
  */
+/*
+ * Lossless exponent-split codec for high-precision pages ("ExANS komprimerer
+ * KV-cache og goer AI-svar hurtigere paa H100 GPU", ainews.dk, on "ExANS -
+ * Lossless KV cache compression at 622 GB/s on H100"): every BF16 value is
+ * split into its exponent and its sign + mantissa; the exponents of a group
+ * are coded with an asymmetric numeral system around the group's centre,
+ * the sign + mantissa bytes are kept raw.  A group is one page of one pool
+ * ([Hkv][16][D] bf16, N = Hkv*16*D values; N <= 2^22), coded on its own:
+ *   - centre = the most frequent exponent (smallest among ties); symbol =
+ *     exponent - centre + 8 when in 0..14, else 15 (escape, its exponent
+ *     byte kept in an escape stream in element order);
+ *   - byte-wise rANS, 32-bit state in [2^23, 2^31), 12-bit frequencies
+ *     f = max(1, count*4096/N) per present symbol with the remainder on the
+ *     largest; 32 interleaved states (state i codes elements 128c + 4i + r,
+ *     r = 0..3) share one byte stream: after each symbol the states below
+ *     2^23 take one byte each in state order, then a second round likewise;
+ *   - a group whose coded blob would exceed 64 + 2N bytes is stored raw.
+ * Blob (little-endian, a multiple of 16 bytes): u32 total, mode (0 raw,
+ * 1 coded), N, centre, escapes, stream bytes; 8 zero bytes; u16 f[16]; then
+ * the 2N raw bytes, or the N sign+mantissa bytes (sign << 7 | mantissa),
+ * the escape bytes and the rANS stream (32 initial states as u32, then the
+ * renormalisation bytes), each zero-padded to 16.
+ */
+
+/* Workspace bytes kvc_exans_encode needs for n pages: n * (4N + 192). */
+KVC_API kvc_status kvc_exans_workspace_size(int n, int page_size, int n_kv_heads, int head_dim,
+                                            size_t* bytes);
+
+/*
+ * kvc_exans_encode - code n pages into blobs stored back to back.
+ *   src_bf16   device bf16 [n_src][Hkv][16][D], 16-byte aligned
+ *   page_ids   device int32 [n] or NULL: blob i codes src page page_ids[i]
+ *   workspace  device, >= kvc_exans_workspace_size bytes, 16-byte aligned
+ *   dst        device, dst_bytes >= n * (64 + 2N) (no blob exceeds its raw
+ *              size plus the header), 16-byte aligned
+ *   offsets    device int64 [n + 1], out: blob i is dst[offsets[i],
+ *              offsets[i+1]); offsets[n] = the coded size
+ * Errors: INVALID_ARG (null or misaligned pointers, n outside 0..2^24,
+ * dst_bytes too small), WORKSPACE, UNSUPPORTED (page_size != 16, head_dim
+ * not 64/128/256, N > 2^22).  Asynchronous on `stream` (three launches:
+ * code into per-page workspace slots, prefix sum of the sizes, compaction);
+ * allocates nothing.
+ */
+KVC_API kvc_status kvc_exans_encode(const void* src_bf16, const int32_t* page_ids, int n, int page_size,
+                                    int n_kv_heads, int head_dim, void* workspace, size_t workspace_bytes,
+                                    void* dst, size_t dst_bytes, int64_t* offsets, kvc_stream_t stream);
+
+/*
+ * kvc_exans_decode - decode blobs back to bf16 pages (bit-exact inverse).
+ *   src, src_bytes  device blobs as kvc_exans_encode wrote them
+ *   offsets    device int64 [n_blobs + 1]
+ *   blob_ids   device int32 [n] or NULL: page i decodes blob blob_ids[i]
+ *   dst_bf16   device bf16 [n][Hkv][16][D], 16-byte aligned
+ *   device_flags  device uint32 word or NULL: OR-ed with 1 (a blob id,
+ *              offset or header that does not fit; that page is left as it
+ *              is) or 2 (a coded stream or escape stream that does not end
+ *              where its header says: corrupt data)
+ * Errors: INVALID_ARG, UNSUPPORTED as above.  Asynchronous; one warp per
+ * page.
+ */
+KVC_API kvc_status kvc_exans_decode(const void* src, size_t src_bytes, const int64_t* offsets, int n_blobs,
+                                    const int32_t* blob_ids, int n, int page_size, int n_kv_heads,
+                                    int head_dim, void* dst_bf16, uint32_t* device_flags,
+                                    kvc_stream_t stream);
+
 KVC_API kvc_status kvc_promote_pages(const kvc_paged_cache* cache, int32_t* block_table,
                                      uint8_t* older_fmt, const int32_t* context_lens,
                                      const int32_t* req_seq, const int32_t* req_page,

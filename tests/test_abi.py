@@ -175,3 +175,38 @@ def test_promote_argument_errors():
     assert call(tags=False) == K.KVC_ERR_INVALID_ARG        # the tag makes a page an anchor
     assert call(ptr=0) == K.KVC_ERR_INVALID_ARG
     assert call(batch=1 << 20, max_pages=1 << 12) == K.KVC_ERR_UNSUPPORTED
+
+
+def test_exans_argument_errors():
+    """Host-side validation of the exponent-split codec entry points (nothing launched)."""
+    import ctypes
+    lib = ctypes.CDLL(K.LIB_PATH)
+    lib.kvc_exans_encode.restype = ctypes.c_int
+    lib.kvc_exans_decode.restype = ctypes.c_int
+    vp = ctypes.c_void_p
+    assert K.kvc_exans_workspace_size(10, 16, 8, 128) == 10 * (4 * 8 * 16 * 128 + 192)
+    with pytest.raises(K.KvcError):
+        K.kvc_exans_workspace_size(1, 8, 8, 128)                  # page size 16 only
+    with pytest.raises(K.KvcError):
+        K.kvc_exans_workspace_size(1, 16, 8, 96)                  # head_dim 64/128/256
+    with pytest.raises(K.KvcError):
+        K.kvc_exans_workspace_size(1, 16, 1 << 12, 256)           # N > 2^22
+    p = vp(1 << 20)
+    N = 8 * 16 * 128
+    ws = 4 * N + 192
+
+    def enc(n=2, ptr=p, ws_bytes=2 * ws, dst_bytes=2 * (64 + 2 * N), d=128):
+        return lib.kvc_exans_encode(ptr, None, n, 16, 8, d, ptr, ctypes.c_size_t(ws_bytes), ptr,
+                                    ctypes.c_size_t(dst_bytes), ptr, None)
+    assert enc(n=-1) == K.KVC_ERR_INVALID_ARG
+    assert enc(d=80) == K.KVC_ERR_UNSUPPORTED
+    assert enc(ptr=None) == K.KVC_ERR_INVALID_ARG
+    assert enc(ptr=vp((1 << 20) + 8)) == K.KVC_ERR_INVALID_ARG   # misaligned
+    assert enc(ws_bytes=2 * ws - 1) == K.KVC_ERR_WORKSPACE
+    assert enc(dst_bytes=2 * (64 + 2 * N) - 16) == K.KVC_ERR_INVALID_ARG
+    def dec(n=2, ptr=p, d=128):
+        return lib.kvc_exans_decode(ptr, ctypes.c_size_t(1 << 20), ptr, 2, None, n, 16, 8, d, ptr, None, None)
+    assert dec(n=0) == K.KVC_OK
+    assert dec(n=-3) == K.KVC_ERR_INVALID_ARG
+    assert dec(d=32) == K.KVC_ERR_UNSUPPORTED
+    assert dec(ptr=None) == K.KVC_ERR_INVALID_ARG
