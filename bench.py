@@ -140,6 +140,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------- our arm
 
+def max_over_ranks(value, world, dev):
+    """Device time of the job: the largest of the ranks' times (every rank
+    takes part in the same collective, so call it on every rank)."""
+    if world <= 1:
+        return value
+    t = torch.tensor([float(value)], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank):
+    """Each rank decodes its own independent batch (weak scaling): inputs are
+    drawn with the rank as the seed."""
+    return rank
+
+
 # the source file that holds each timed kernel
 KERNEL_FILE = {"decode": "decode_tc.cu", "pack_ternary": "quant.cu", "pack_fp8": "quant.cu",
                "pack_bf16": "quant.cu", "pack": "quant.cu", "dequant": "quant.cu"}
@@ -178,7 +194,7 @@ def run_ours(args, rank, world, dev, peak, peak_src):
     from compressed_decode_attention_kvc_b200 import paged_cache as PC
 
     n_layers = layers_of(args)
-    inp = synth.make_decode_inputs(args.workload, seed=rank, device=dev, batch=args.batch)
+    inp = synth.make_decode_inputs(args.workload, seed=rank_seed(rank), device=dev, batch=args.batch)
     cfg = inp["cfg"]
     B, max_pages, H, _, D = inp["k_pages"].shape
     if n_layers > 1:
@@ -295,10 +311,7 @@ def run_ours(args, rank, world, dev, peak, peak_src):
         raise RuntimeError(f"device error flags {flags}")
 
     step_bytes = sum(nbytes.values())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
     value = step_bytes * world * args.steps / (total_ms * 1e-3) / 1e9
 
@@ -632,10 +645,7 @@ def run_e2e(args, K, PC, inp, cfg, layout, cache, kf, vf, older, ws, ws_bytes, o
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     h2d = (hk.numel() * 2 + hv.numel() * 2 + hq_t.numel() * 2 + hl.numel() * 4
            + layout.block_table.numel() * 4 + n_layers * sum(len(x) for x in layout.pool_src_ids) * 4)
     return {"value": step_bytes * world * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -654,7 +664,7 @@ def run_bulk(args, rank, world, dev, peak, peak_src):
     """One step = ternary quantise+pack of every page of the 1 GiB workload,
     then dequantise all of it back to bf16 (both directions timed)."""
     import compressed_decode_attention_kvc_b200 as K
-    pages = synth.make_bulk_pages(seed=rank, device=dev)              # [n][H][P][D] bf16
+    pages = synth.make_bulk_pages(seed=rank_seed(rank), device=dev)              # [n][H][P][D] bf16
     n, H, _, D = pages.shape
     codes = torch.empty((n, H, P, D // 4), dtype=torch.uint8, device=dev)
     gamma = torch.empty((n, H), dtype=torch.float32, device=dev)
@@ -716,10 +726,7 @@ def run_bulk(args, rank, world, dev, peak, peak_src):
     total_ms = t0.elapsed_time(t1)
     del graph
     step_bytes = sum(nbytes.values())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     kernels = {}
     for name, ts in per_kernel.items():
         avg = sum(ts) / len(ts)
@@ -766,10 +773,7 @@ def run_bulk(args, rank, world, dev, peak, peak_src):
         b.record(stream)
         torch.cuda.synchronize()
         ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = max_over_ranks(ms, world, dev)
         res["e2e"] = {"value": step_bytes * world * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
                       "h2d_bytes_per_step": int(pages.numel() * 2), "d2h_bytes_per_step": int(rt.numel() * 2),
                       "ms_per_step": ms / steps, "steps": steps}
@@ -883,7 +887,9 @@ def run_reference(args):
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_block(args, cfg),
+            "data": "synthetic",
+            # the workload our arm runs; the sample drawn from it is in cpu_baseline
+            "config": config_block(args, dict(cfg, batch=args.batch or synth.WORKLOADS[args.workload]["batch"])),
             "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
