@@ -424,37 +424,49 @@ __device__ __noinline__ void merge_partials(MergeArgs p, int bg, int rec0, int r
       ls[r] += lk;
     }
   }
-  // output rows: lane owns D/32 consecutive dims of every row
+  // output rows: lane owns D/32 consecutive dims of every row.  Records are
+  // the outer loop, so the loads of all rows of a record (and of the next
+  // record) are independent and in flight together.
   constexpr int DPL = D / 32;
+  float o[8][DPL];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    if (r >= G) break;
-    float o[DPL];
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) o[i] = 0.f;
-    if (ms[r] != -INFINITY) {
-      for (int k0 = 0; k0 < nrec; k0 += 32) {
-        const int k = k0 + lane;
-        float f = 0.f;
-        if (k < nrec) f = ex2(__ldcg(p.partials + (long long)(rec0 + k * rstride) * rs + r * (D + 2)) - ms[r]);
-        const int kn = min(32, nrec - k0);
-#pragma unroll 4
-        for (int kk = 0; kk < kn; ++kk) {
-          const float fk = __shfl_sync(kFull, f, kk);
-          const float* row = p.partials + (long long)(rec0 + (k0 + kk) * rstride) * rs + r * (D + 2) + 2 + lane * DPL;
+    for (int i = 0; i < DPL; ++i) o[r][i] = 0.f;
+  for (int k0 = 0; k0 < nrec; k0 += 32) {
+    const int k = k0 + lane;
+    float f[8];                                  // weight of record k in each row
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      f[r] = 0.f;
+      if (r < G && k < nrec && ms[r] != -INFINITY)
+        f[r] = ex2(__ldcg(p.partials + (long long)(rec0 + k * rstride) * rs + r * (D + 2)) - ms[r]);
+    }
+    const int kn = min(32, nrec - k0);
+#pragma unroll 2
+    for (int kk = 0; kk < kn; ++kk) {
+      const float* base = p.partials + (long long)(rec0 + (k0 + kk) * rstride) * rs + 2 + lane * DPL;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float fk = __shfl_sync(kFull, f[r], kk);
+        if (r < G) {
 #pragma unroll
           for (int i = 0; i < DPL; i += 2) {
-            const float2 v = __ldcg(reinterpret_cast<const float2*>(row + i));
-            o[i] = fmaf(fk, v.x, o[i]);
-            o[i + 1] = fmaf(fk, v.y, o[i + 1]);
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(base + r * (D + 2) + i));
+            o[r][i] = fmaf(fk, v.x, o[r][i]);
+            o[r][i + 1] = fmaf(fk, v.y, o[r][i + 1]);
           }
         }
       }
     }
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r >= G) break;
     const float inv = ls[r] > 0.f ? 1.f / ls[r] : 0.f;
     float* dst = p.out + ((long long)b * p.Hq + g * G + r) * D + lane * DPL;
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) dst[i] = o[i] * inv;
+    for (int i = 0; i < DPL; ++i) dst[i] = o[r][i] * inv;
   }
   if (lane == 0) p.tickets[bg] = 0u;
 }

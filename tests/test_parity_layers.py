@@ -79,3 +79,77 @@ def test_layers_match_oracle_per_layer(cuda_device, name, over, n_layers):
 def test_layers_large_virtual_batch_cuda_core_kernel(cuda_device):
     # layers * batch above the tensor-core kernel's batch limit (1024)
     _run("tiny", dict(batch=260, context=64, window=16), 4, cuda_device)
+
+
+def test_qwen3b_36_layers_full_size_sampled(cuda_device):
+    """The launch the benchmark times for the Qwen2.5-3B-shaped workload: 36
+    layers of the full-size layer (B = 8, L = 4096) packed by the library and
+    decoded in one launch.  For sampled (layer, sequence) pairs the library's
+    pages are checked against the oracle's codec and then replaced by the
+    oracle's bytes; those rows must match the oracle's attention.  Every row
+    is finite and a convex combination of its layer's values."""
+    from compressed_decode_attention_kvc_b200 import paged_cache as PC
+    from kvc_testlib import check_ternary
+    dev = cuda_device
+    n_layers, P = 36, 16
+    inps = [synth.make_decode_inputs("qwen3b", seed=1000 + l, device=dev) for l in range(n_layers)]
+    cfg = inps[0]["cfg"]
+    hp = HP[cfg["hp"]]
+    B, max_pages, hkv, _, D = inps[0]["k_pages"].shape
+    hq = cfg["n_q_heads"]
+    lens_h = inps[0]["context_lens"].cpu()
+    layout = PC.plan_paged_cache(lens_h, max_pages, cfg["sink"], cfg["window"], hp)
+    cache = PC.allocate_device_cache(layout, hkv, D, dev, n_layers=n_layers)
+    kf = torch.cat([i["k_pages"] for i in inps]).view(n_layers * B * max_pages, hkv, P, D)
+    vf = torch.cat([i["v_pages"] for i in inps]).view(n_layers * B * max_pages, hkv, P, D)
+    PC.compress_into(cache, kf, vf)
+    torch.cuda.synchronize()
+    bt, pf = layout.block_table.numpy(), layout.page_fmt.numpy()
+    per_layer = layout.pool_pages
+    pools = cache.pools
+    refs = {}
+    for l, b in [(0, 0), (17, 5), (35, 7)]:
+        L = int(lens_h[b])
+        sub = {"k_pages": inps[l]["k_pages"][b:b + 1].cpu(), "v_pages": inps[l]["v_pages"][b:b + 1].cpu(),
+               "context_lens": lens_h[b:b + 1], "anchor": inps[l]["anchor"][b:b + 1].cpu(), "slot_key": None,
+               "cfg": cfg}
+        oc, obt, ofmt, _ = oracle_build_from_inputs(sub, hp)
+        npg = O.num_pages(L)
+        assert np.array_equal(ofmt[0, :npg], pf[b, :npg])
+        for f, (kn, vn, ks, vs) in ((O.FP8_E4M3, ("k_fp8", "v_fp8", "k_fp8_scale", "v_fp8_scale")),
+                                    (O.TERNARY, ("k_tern", "v_tern", "k_gamma", "v_gamma"))):
+            js = np.nonzero(pf[b, :npg] == f)[0]
+            if len(js) == 0:
+                continue
+            gslots = torch.from_numpy(l * per_layer[f] + bt[b, js].astype(np.int64)).to(dev)
+            oslots = obt[0, js]
+            for nm, sn, src in ((kn, ks, kf), (vn, vs, vf)):
+                o_pool = getattr(oc, nm)[oslots]
+                if f == O.TERNARY:
+                    rows = torch.from_numpy(((l * B + b) * max_pages + js).astype(np.int64)).to(dev)
+                    check_ternary(pools[nm][gslots].cpu().numpy(), pools[sn][gslots].cpu().numpy(),
+                                  bits(src[rows]))
+                else:
+                    assert np.array_equal(pools[nm][gslots].cpu().numpy(), o_pool)
+                    assert np.array_equal(pools[sn][gslots].cpu().numpy(), getattr(oc, sn)[oslots])
+                pools[nm][gslots] = torch.from_numpy(o_pool).to(dev)
+                pools[sn][gslots] = torch.from_numpy(getattr(oc, sn)[oslots]).to(dev)
+        refs[(l, b)] = O.decode_attention(bits(inps[l]["q"][b:b + 1]), oc, obt, ofmt, [L], hkv)[0]
+
+    q = torch.cat([i["q"] for i in inps])                       # [layers * B][Hq][D]
+    ws_bytes = K.kvc_decode_workspace_size(n_layers * B, hq, hkv, D, max_pages)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.full((n_layers * B, hq, D), float("nan"), device=dev)
+    K.kvc_decode_attention_paged_layers(q, cache.struct, cache.block_table, None, inps[0]["context_lens"],
+                                        n_layers, B, hq, hkv, D, P, max_pages, cfg["sink"], cfg["window"], hp,
+                                        0.0, out, ws, ws_bytes)
+    assert K.kvc_decode_read_error(ws, n_layers * B, hq, hkv, D, max_pages) == 0
+    out_h = out.cpu().numpy().reshape(n_layers, B, hq, D)
+    for (l, b), ref in refs.items():
+        assert_attention_close(out_h[l, b], ref, f"qwen3b layer {l} b={b}")
+    assert np.isfinite(out_h).all()
+    G = hq // hkv
+    for l in range(n_layers):
+        vmax = inps[l]["v_pages"].abs().amax(dim=(1, 3, 4)).float().cpu().numpy()     # [B][Hkv]
+        bound = np.repeat(vmax, G, axis=1)[:, :, None] * (1 + 1e-3) + 1e-6
+        assert np.all(np.abs(out_h[l]) <= bound), l
