@@ -67,7 +67,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kCostTern = 4, kCostMax = 24;
 template <int D, bool NARROW>
 __host__ __device__ constexpr int cost_hp(int fmt) {
-  return fmt == KVC_FMT_BF16 ? (D == 256 ? 21 : (NARROW ? 16 : 22)) : 9;
+  return fmt == KVC_FMT_BF16 ? (D == 256 ? 21 : (NARROW ? 16 : 22)) : (NARROW || D == 256 ? 9 : 16);
 }
 
 struct Desc {
