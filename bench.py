@@ -156,19 +156,47 @@ def rank_seed(rank):
     return rank
 
 
-# the source file that holds each timed kernel
-KERNEL_FILE = {"decode": "decode_tc.cu", "pack_ternary": "quant.cu", "pack_fp8": "quant.cu",
-               "pack_bf16": "quant.cu", "pack": "quant.cu", "dequant": "quant.cu"}
+# where each timed kernel's code lives: (file, kernel function, launcher);
+# None = the whole file
+KERNEL_SRC = {"decode": ("decode_tc.cu", None, None),
+              "pack_ternary": ("quant.cu", "quant_ternary_kernel", "launch_quant_ternary"),
+              "pack": ("quant.cu", "quant_ternary_kernel", "launch_quant_ternary"),
+              "dequant_ternary": ("quant.cu", "dequant_ternary_kernel", "launch_dequant_ternary")}
+
+
+def _function_text(src, name, start_at_file_head):
+    """Text of the definition of `name` (to its closing brace at column 0);
+    with start_at_file_head, everything before it too (the helpers it uses)."""
+    i = src.find(" " + name + "(")
+    if i < 0:
+        return None
+    j = src.find("\n}\n", i)
+    if j < 0:
+        return None
+    start = 0 if start_at_file_head else src.rfind("\n", 0, i) + 1
+    return src[start:j + 3]
 
 
 def kernel_source_hash(kernel_key):
-    """Hash of the source file holding the kernel: recorded ncu traffic
-    stays valid only while that file is unchanged."""
-    f = KERNEL_FILE.get(kernel_key)
-    if f is None:
+    """Hash of the code of a kernel: recorded ncu traffic stays valid only
+    while that code is unchanged.  For a codec kernel that is the source
+    file up to the end of the kernel (the helpers it uses come first) plus
+    its launcher; for decode, the whole file."""
+    spec = KERNEL_SRC.get(kernel_key)
+    if spec is None:
         return None
+    f, fn, launcher = spec
     path = os.path.join(ROOT, "compressed_decode_attention_kvc_b200", "csrc", f)
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    src = open(path).read()
+    if fn is None:
+        text = src
+    else:
+        a = _function_text(src, fn, True)
+        b = _function_text(src, launcher, False)
+        if a is None or b is None:
+            return None
+        text = a + b
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
 def ncu_traffic(kernel_key, workload):

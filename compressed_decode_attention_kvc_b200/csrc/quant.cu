@@ -160,6 +160,64 @@ __global__ void __launch_bounds__(256) quant_fp8_kernel(const uint4* __restrict_
   if (threadIdx.x == 0) scale[i] = sc;
 }
 
+// Single-pass FP8 page quantise for pages of WPP * 32 * CPL chunks (16 B
+// each): WPP warps per page, CPL chunks per lane held in registers, so the
+// page is read from DRAM once and never re-read; 8 / WPP pages per CTA.  The amax
+// is a warp reduction (and a shared-memory one across the page's warps);
+// the encode is the same float32 arithmetic as quant_fp8_kernel.
+template <int WPP, int CPL>
+__global__ void __launch_bounds__(256, 3) quant_fp8_reg_kernel(const uint4* __restrict__ src,
+                                                            const int32_t* __restrict__ page_ids, int n,
+                                                            uint2* __restrict__ dst, float* __restrict__ scale) {
+  constexpr int CPP = WPP * 32 * CPL;        // chunks per page
+  __shared__ float red[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int part = warp % WPP;
+  const long long i = (long long)blockIdx.x * (8 / WPP) + warp / WPP;
+  const bool valid = i < n;
+  uint4 v[CPL];
+  float amax = 0.f;
+  if (valid) {
+    const long long sp = page_ids ? (long long)page_ids[i] : i;
+    const uint4* s = src + sp * CPP + part * (32 * CPL);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) v[c] = ld_stream(s + c * 32 + lane);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  }
+  if constexpr (WPP > 1) {
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    const int w0 = warp - part;
+#pragma unroll
+    for (int k = 0; k < WPP; ++k) amax = fmaxf(amax, red[w0 + k]);
+  }
+  if (!valid) return;
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
+  uint2* d = dst + i * CPP + part * (32 * CPL);
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 y = make_float2(__fmul_rn(bf16_lo(w[k]), inv), __fmul_rn(bf16_hi(w[k]), inv));
+      const uint32_t e2 = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);  // .x -> low byte
+      packed[k >> 1] |= e2 << (16 * (k & 1));
+    }
+    d[c * 32 + lane] = make_uint2(packed[0], packed[1]);
+  }
+  if (lane == 0 && part == 0) scale[i] = sc;
+}
+
 __global__ void __launch_bounds__(256) copy_pages_kernel(const uint4* __restrict__ src,
                                                          const int32_t* __restrict__ page_ids,
                                                          long long n_chunks, long long cpp,
@@ -621,8 +679,19 @@ cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, int n
 cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, int n, int hkv, int d,
                              void* dst, float* scale, cudaStream_t s) {
   const int cpp = hkv * kPage * d / 8;
-  quant_fp8_kernel<<<n, 256, 0, s>>>(static_cast<const uint4*>(src), page_ids, cpp,
-                                      static_cast<uint2*>(dst), scale);
+  auto* in = static_cast<const uint4*>(src);
+  auto* out = static_cast<uint2*>(dst);
+  // pages of 512, 1024, 2048 or 4096 chunks (Hkv * D = 256 .. 2048): the
+  // register-resident kernel; other sizes: the two-pass one
+  switch (cpp) {
+    // (measured: 4 warps x 4 chunks per lane for 8 KB pages and 8 x 8 for
+    // 32 KB pages beat 2 x 8 / 8 x 2 and 4 x 16)
+    case 512: quant_fp8_reg_kernel<4, 4><<<grid_for(n, 2), 256, 0, s>>>(in, page_ids, n, out, scale); break;
+    case 1024: quant_fp8_reg_kernel<4, 8><<<grid_for(n, 2), 256, 0, s>>>(in, page_ids, n, out, scale); break;
+    case 2048: quant_fp8_reg_kernel<8, 8><<<n, 256, 0, s>>>(in, page_ids, n, out, scale); break;
+    case 4096: quant_fp8_reg_kernel<8, 16><<<n, 256, 0, s>>>(in, page_ids, n, out, scale); break;
+    default: quant_fp8_kernel<<<n, 256, 0, s>>>(in, page_ids, cpp, out, scale); break;
+  }
   return cudaGetLastError();
 }
 

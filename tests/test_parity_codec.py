@@ -79,7 +79,7 @@ def test_page_ids_gather_and_order(cuda_device):
             assert torch.equal(sub_s.cpu(), full_s.cpu()[idx])
 
 
-@pytest.mark.parametrize("d,hkv", [(64, 4), (128, 2), (128, 8), (256, 4)])
+@pytest.mark.parametrize("d,hkv", [(64, 4), (128, 2), (128, 4), (128, 8), (256, 4), (256, 8), (64, 3), (64, 1)])
 def test_fp8_quantize_bit_exact(cuda_device, d, hkv):
     src = _rand_pages(29, hkv, d, seed=d + hkv, dev=cuda_device, dist="outlier")
     src[3].zero_()
