@@ -68,6 +68,8 @@ struct EncSmem {
   uint32_t hist[256];   // exponent histogram
   uint32_t cnt[16];     // symbol counts
   uint32_t fc[16];      // f | cum << 16
+  uint32_t rcp[16];     // x / f = umulhi(x, rcp) >> rsh for x < 2^31 (f >= 2)
+  uint32_t rsh[16];
 };
 
 // One warp per group; the group's blob is built in its workspace slot of
@@ -165,6 +167,14 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint1
     for (int t = 0; t < 16; ++t) {
       S.fc[t] = (uint32_t)f[t] | (cum << 16);
       cum += (uint32_t)f[t];
+      // division by the frequency as a multiply (Granlund and Montgomery's
+      // round-up reciprocal): with l = ceil(log2 f) and m = ceil(2^(31+l) / f)
+      // < 2^32, floor(x / f) = floor(x * m / 2^(31+l)) for every x < 2^31,
+      // since the rounding adds less than x / 2^(31+l) < 1/f
+      const uint32_t fu = (uint32_t)f[t];
+      const int l = fu > 1u ? 32 - __clz(fu - 1u) : 0;
+      S.rcp[t] = fu > 1u ? (uint32_t)(((1ull << (31 + l)) + fu - 1u) / fu) : 0u;
+      S.rsh[t] = fu > 1u ? (uint32_t)(l - 1) : 0u;
     }
   }
   __syncwarp();
@@ -201,7 +211,9 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint1
         st >>= 8;
         nb = 2;
       }
-      st = ((st / f) << kExScaleBits) + (st % f) + cum;
+      // (st / f) << 12 + st % f + cum, with st < f * 2^19 <= 2^31 here
+      const uint32_t q = f == 1u ? st : (__umulhi(st, S.rcp[s]) >> S.rsh[s]);
+      st = st + cum + q * (kExM - f);
       const unsigned b1 = __ballot_sync(kFull, nb >= 1), b2 = __ballot_sync(kFull, nb == 2);
       const int n1 = __popc(b1), n2 = __popc(b2);
       written += n1 + n2;
