@@ -723,3 +723,27 @@ def test_promote_keeps_attention_when_values_are_exact(anchor_fmt):
     assert all(fmt2[b, j] == anchor_fmt for b, j in pick)
     got = O.decode_attention(q, out, bt2, fmt2, lens, hkv)
     assert np.abs(got - ref).max() < (1e-12 if anchor_fmt == O.BF16 else 1e-6)
+
+
+def test_promote_fp8_within_e4m3_rounding_of_the_stale_values():
+    """An FP8 anchor decodes (s * e) to the stale page's bf16(gamma * c)
+    within half an e4m3 step: relative 2^-4 for normal e4m3 values, and the
+    head with the largest gamma maps to +-448 exactly."""
+    rng = np.random.default_rng(31)
+    hkv, d = 4, 16
+    codes = rng.choice(np.array([0x55, 0xFF, 0x1D, 0x00, 0x7D], np.uint8), size=(hkv, 16, d // 4))
+    codes[0] = 0x55                                          # head 0: all +1
+    gam = np.float32([2.5, 0.37, 0.011, 1.9])
+    cache, bt, tags = _one_stale_page_cache(codes, gam, d=d)
+    out, _, _, _, flags = O.promote_pages(cache, bt, tags, [40], [0], [1], [0], 4, 8, O.BF16, O.FP8_E4M3)
+    assert flags == 0
+    want = O.bf16_to_f64(O.dequantize_ternary(codes[None], gam[None])[0])          # [Hkv][P][D]
+    got = float(out.k_fp8_scale[0]) * O.e4m3_to_f64(out.k_fp8[0])
+    amax = np.abs(want).max()
+    assert np.all(np.abs(out.k_fp8[0][0]) == 0x7E)                  # +448 (the largest gamma is head 0)
+    nz = want != 0
+    assert np.all(np.sign(got[nz]) == np.sign(want[nz])) and np.all(got[~nz] == 0)
+    normal = np.abs(want) >= amax / 448 * 2.0 ** -6                # e4m3 normal range after scaling
+    assert np.all(np.abs(got - want)[normal] <= np.abs(want)[normal] * 2.0 ** -4 + 1e-12)
+    sub = nz & ~normal
+    assert np.all(np.abs(got - want)[sub] <= amax / 448 * 2.0 ** -10 + 1e-12)   # half a subnormal step
