@@ -72,3 +72,28 @@ def test_bench_traffic_records_follow_the_kernel_code(tmp_path):
         assert rec > 0
     assert bench.ncu_traffic("decode", None) is None
     assert bench.ncu_traffic("decode", "no_such_workload") is None
+
+
+def test_bench_algorithmic_bytes_match_the_storage_accounting():
+    """The roofline numerator: bytes each kernel of a step must move, from
+    the oracle's storage accounting (pinned to the pages' figures)."""
+    import oracle as O
+    bench = _bench()
+    lens = torch.tensor([16 * 9 + 3, 16 * 4, 200], dtype=torch.int32)
+    max_pages = 16
+    cfg = dict(n_kv_heads=4, head_dim=128, n_q_heads=16)
+    H, D, hq, P = 4, 128, 16, 16
+    lay = PC.plan_paged_cache(lens, max_pages, 4, 40, K.KVC_FMT_FP8_E4M3)
+    n_bf, n_f8, n_t = lay.pool_pages
+    got = bench.algorithmic_bytes(cfg, lay, 3, max_pages, has_older=False)
+    bf16_page = 2 * P * H * D
+    tern_page = H * O.ternary_group_bytes(P, D)                 # codes + one gamma per head
+    fp8_page = O.fp8_page_bytes(P, H, D)
+    assert got["pack_ternary"] == 2 * n_t * (bf16_page + tern_page)
+    assert got["pack_fp8"] == 2 * n_f8 * (bf16_page + fp8_page)
+    assert got["pack_bf16"] == 2 * n_bf * 2 * bf16_page
+    pages = n_bf + n_f8 + n_t
+    per_seq = 2 * hq * D + 4 * hq * D + 4                       # Q bf16, out fp32, length
+    assert got["decode"] == 2 * (n_bf * bf16_page + n_f8 * fp8_page + n_t * tern_page) + 3 * per_seq + 4 * pages
+    tagged = bench.algorithmic_bytes(cfg, lay, 3, max_pages, has_older=True)
+    assert tagged["decode"] == got["decode"] + pages               # one tag byte per page
