@@ -96,6 +96,8 @@ const char* kvc_status_string(kvc_status status) {
   return "unknown status";
 }
 
+int kvc_layout_version(void) { return KVC_LAYOUT_VERSION; }
+
 kvc_status kvc_quantize_pack_pages(const void* src_bf16, const int32_t* page_ids, int n,
                                    int page_size, int n_kv_heads, int head_dim, kvc_format mode,
                                    void* dst, float* dst_scale, kvc_stream_t stream) {

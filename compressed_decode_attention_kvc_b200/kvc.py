@@ -31,6 +31,7 @@ KVC_FMT_FP8_E4M3 = 1
 KVC_FMT_TERNARY2 = 2
 
 PAGE_SIZE = 16
+LAYOUT_VERSION = 1             # KVC_LAYOUT_VERSION of include/kvc.h
 
 # device error flags returned by kvc_decode_read_error
 ERR_BLOCK_TABLE = 1
@@ -43,7 +44,7 @@ EXPORTS = (
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
     "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc", "kvc_append_retier",
     "kvc_decode_attention_paged_layers", "kvc_promote_pages", "kvc_exans_workspace_size",
-    "kvc_exans_encode", "kvc_exans_decode",
+    "kvc_exans_encode", "kvc_exans_decode", "kvc_layout_version",
 )
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -75,6 +76,8 @@ def _load() -> ctypes.CDLL:
     vp, i32, f32, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int
     lib.kvc_status_string.restype = ctypes.c_char_p
     lib.kvc_status_string.argtypes = [st]
+    lib.kvc_layout_version.restype = ctypes.c_int
+    lib.kvc_layout_version.argtypes = []
     lib.kvc_quantize_pack_pages.restype = st
     lib.kvc_quantize_pack_pages.argtypes = [vp, vp, i32, i32, i32, i32, st, vp, vp, vp]
     lib.kvc_dequantize_pages.restype = st
@@ -182,6 +185,11 @@ def kvc_promote_pages(cache: kvc_paged_cache, block_table, older_fmt, context_le
                                   n_kv_heads, head_dim, page_size, max_pages, sink_tokens, window_tokens,
                                   hp_mode, anchor_fmt, _stream(stream)),
            "kvc_promote_pages")
+
+
+def kvc_layout_version() -> int:
+    """Byte-layout version of the loaded library (include/kvc.h, KVC_LAYOUT_VERSION)."""
+    return int(_lib.kvc_layout_version())
 
 
 def kvc_exans_workspace_size(n, page_size, n_kv_heads, head_dim) -> int:

@@ -77,8 +77,24 @@ typedef enum {
 
 #define KVC_PAGE_SIZE 16
 
+/*
+ * Version of the byte layouts the library writes and reads; compressed
+ * pages are persistent data (saved, offloaded, reloaded), so a layout
+ * change bumps it.  Version 1:
+ *   ternary group  [Hkv][16][D/4] bytes per page, element i of a group's
+ *                  row-major [token][dim] order at byte i/4, bits 2(i%4)..+1,
+ *                  fields 00 = 0, 01 = +1, 11 = -1; gamma fp32 [Hkv] per page
+ *   FP8 page       [Hkv][16][D] OCP e4m3 bytes + one fp32 scale per page
+ *   BF16 page      [Hkv][16][D] bf16
+ *   codec blob     as described above kvc_exans_encode
+ */
+#define KVC_LAYOUT_VERSION 1
+
 /* Human-readable name of a status code (static string, never NULL). */
 KVC_API const char* kvc_status_string(kvc_status status);
+
+/* KVC_LAYOUT_VERSION of the library as built (compare with the header's). */
+KVC_API int kvc_layout_version(void);
 
 /*
  * kvc_quantize_pack_pages - compress whole pages into one page format.

@@ -210,3 +210,9 @@ def test_exans_argument_errors():
     assert dec(n=-3) == K.KVC_ERR_INVALID_ARG
     assert dec(d=32) == K.KVC_ERR_UNSUPPORTED
     assert dec(ptr=None) == K.KVC_ERR_INVALID_ARG
+
+
+def test_layout_version_matches_the_header():
+    src = open(os.path.join(ROOT, "include", "kvc.h")).read()
+    v = int(re.search(r"#define KVC_LAYOUT_VERSION (\d+)", src).group(1))
+    assert K.kvc_layout_version() == v == K.LAYOUT_VERSION
