@@ -127,3 +127,40 @@ def test_pages_round_trip():
     assert off[0] == 0 and off[-1] == len(pool) and (np.diff(off) % 16 == 0).all()
     back = X.decode_pages(pool, off, (2, 16, 64))
     assert np.array_equal(back, pages[[4, 0, 2]])
+
+
+def test_rans_round_trip_on_adversarial_tables():
+    """The coder on its own, with tables the exponent data rarely produces:
+    symbols of frequency 1 used often (two renormalisation bytes per
+    symbol), a table of one symbol, and uniform tables.  Decoding gives
+    the symbols back and the size stays at the cross-entropy."""
+    rng = np.random.default_rng(9)
+    n = 4096
+    cases = []
+    f = np.zeros(16, np.int64); f[0] = 1; f[1] = 1; f[2] = X.M - 2
+    cases.append((rng.choice([0, 1, 2], size=n, p=[0.45, 0.45, 0.10]), f))          # rare-by-table symbols dominate
+    f = np.zeros(16, np.int64); f[7] = X.M
+    cases.append((np.full(n, 7), f))                                                 # one symbol
+    cases.append((rng.integers(0, 16, n), np.full(16, X.M // 16, np.int64)))         # uniform, 4 bits each
+    f = np.full(16, 1, np.int64); f[15] = X.M - 15
+    cases.append((rng.integers(0, 15, n), f))                                        # 15 symbols at 1/4096
+    for sym, f in cases:
+        assert f.sum() == X.M and (f[np.unique(sym)] > 0).all()
+        stream = X.rans_encode(sym, f)
+        assert np.array_equal(X.rans_decode(stream, f, n), sym)
+        bits = float(sum(-math.log2(f[s] / X.M) for s in sym))
+        assert bits / 8 - 4 <= len(stream) <= bits / 8 + 32 * 5, (len(stream), bits / 8)
+
+
+def test_normalise_properties():
+    rng = np.random.default_rng(10)
+    for _ in range(300):
+        n = int(rng.integers(128, 1 << 16)) // 128 * 128 or 128
+        k = int(rng.integers(1, 17))
+        probs = rng.dirichlet(np.full(k, float(rng.choice([0.05, 1.0, 20.0]))))
+        counts = np.zeros(16, np.int64)
+        idx = rng.choice(16, size=k, replace=False)
+        counts[idx] = rng.multinomial(n, probs)
+        f = X.normalise(counts, n)
+        assert f.sum() == X.M
+        assert np.array_equal(f > 0, counts > 0) and (f >= 0).all()
