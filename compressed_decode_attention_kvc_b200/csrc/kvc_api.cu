@@ -3,6 +3,8 @@
 // allocates memory or synchronises (except kvc_decode_read_error, whose job
 // is to read a device flag).
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <algorithm>
 #include <vector>
@@ -35,19 +37,44 @@ kvc_status check_codec(const void* src, const void* dst, int n, int page_size, i
 
 namespace kvc {
 
+// The tensor-memory (tcgen05) decode kernel is the alternative
+// implementation, measured slower than the register-sourced one on every
+// workload here; it runs only when the environment variable
+// KVC_DECODE_KERNEL is "tcgen05" (read once per process).
+static bool umma_selected() {
+  static const bool on = [] {
+    const char* v = getenv("KVC_DECODE_KERNEL");
+    return v != nullptr && strcmp(v, "tcgen05") == 0;
+  }();
+  return on;
+}
+
 cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, DecodePlan* plan) {
   const long long bg = (long long)batch * hkv;
   const int G = hq / hkv;
   const size_t record = (size_t)G * (d + 2) * sizeof(float);
   plan->ticket_offset = 256;
   plan->partial_offset = round_up(256 + (size_t)bg * 4, 256);
+  if (umma_selected() && umma_supported(batch, d, hkv, max_pages)) {
+    // persistent grid, one CTA of two warpgroup workers per SM; two records
+    // (ternary, high precision) per (worker, pair) boundary
+    int grid = 0;
+    cudaError_t e = umma_grid(batch, d, hq, hkv, &grid);
+    if (e != cudaSuccess) return e;
+    plan->kernel = kDecodeUmma;
+    plan->grid = grid;
+    plan->n_splits = 2 * grid * umma_heads_per_cta(hkv);   // two warpgroup workers per CTA
+    plan->pages_per_split = 0;
+    plan->bytes = plan->partial_offset + 2 * ((size_t)plan->n_splits + (size_t)bg) * record;
+    return cudaSuccess;
+  }
   if (tc_supported(batch, hkv, max_pages)) {
     // persistent grid, every warp a stream-K worker; one partial state per
     // (warp, pair) boundary: at most warps + pairs records
     int grid = 0;
     cudaError_t e = tc_grid(batch, d, hq, hkv, &grid);
     if (e != cudaSuccess) return e;
-    plan->tensor_cores = true;
+    plan->kernel = kDecodeTc;
     plan->grid = grid;
     plan->n_splits = grid * tc_warps_per_cta(hkv);
     plan->pages_per_split = 0;
@@ -66,7 +93,7 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
   splits = std::max(1ll, std::min(splits, max_splits));
   const int pps = max_pages > 0 ? (int)((max_pages + splits - 1) / splits) : 1;
   splits = max_pages > 0 ? (max_pages + pps - 1) / pps : 1;
-  plan->tensor_cores = false;
+  plan->kernel = kDecodeSimple;
   plan->grid = 0;
   plan->n_splits = (int)splits;
   plan->pages_per_split = pps;
@@ -75,7 +102,8 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const DecodePlan& plan, cudaStream_t s) {
-  if (plan.tensor_cores) return launch_decode_tc(p, head_dim, plan.grid, s);
+  if (plan.kernel == kDecodeUmma) return launch_decode_umma(p, head_dim, plan.grid, s);
+  if (plan.kernel == kDecodeTc) return launch_decode_tc(p, head_dim, plan.grid, s);
   return launch_decode_simple(p, head_dim, s);
 }
 

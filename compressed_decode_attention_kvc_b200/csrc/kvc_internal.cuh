@@ -81,12 +81,14 @@ struct DecodeParams {
 };
 
 struct DecodePlan {
-  bool tensor_cores;         // decode_tc kernel (else decode_simple)
+  int kernel;                // kDecodeSimple, kDecodeTc or kDecodeUmma
   int n_splits;              // simple: splits per (sequence, KV head); tc: warps in the grid
   int pages_per_split;       // simple only
   int grid;                  // tc only: persistent CTAs
   size_t ticket_offset, partial_offset, bytes;
 };
+
+constexpr int kDecodeSimple = 0, kDecodeTc = 1, kDecodeUmma = 2;
 
 // Kernel choice, split-K plan and workspace layout for these shapes on the
 // current device.
@@ -100,5 +102,12 @@ bool tc_supported(int batch, int hkv, int max_pages);
 cudaError_t tc_grid(int batch, int d, int hq, int hkv, int* grid);
 int tc_warps_per_cta(int hkv);
 cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s);
+
+// tensor-memory (tcgen05) kernel (decode_umma.cu): two partial records per
+// (CTA, sequence, KV head)
+bool umma_supported(int batch, int d, int hkv, int max_pages);
+int umma_heads_per_cta(int hkv);
+cudaError_t umma_grid(int batch, int d, int hq, int hkv, int* grid);
+cudaError_t launch_decode_umma(const DecodeParams& p, int head_dim, int grid, cudaStream_t s);
 
 }  // namespace kvc
