@@ -128,6 +128,24 @@ __device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// bf16 x bf16 -> f32, m16n8k16 (BF16 pages: K, V and Q in their given form)
+__device__ __forceinline__ void mma16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// y as a bf16 pair (hi, lo) with hi = bf16(y), lo = bf16(y - hi): ~16 bits.
+__device__ __forceinline__ uint32_t split_bf16x2(float y) {
+  const float hi = __bfloat162float(__float2bfloat16_rn(y));
+  return bf16x2(hi, y - hi);
+}
+
 // Ternary fields at bit offset o (even, 0..14) of both 16-bit halves -> f16
 // pair of 2*code: 01 -> 0x4000 (+2), 11 -> 0xC000 (-2), 00 -> 0 (10 -> -0).
 __device__ __forceinline__ uint32_t tern2(uint32_t w, int o) {

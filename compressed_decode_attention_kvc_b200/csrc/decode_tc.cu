@@ -103,7 +103,7 @@ struct Worker {
   const DecodeParams& p;
   const Prologue& pr;
   unsigned char* ring;     // the CTA's kEntries slots
-  uint32_t* qsm;           // this warp's f16 Q fragments: [kSteps / 2][32 lanes][4]
+  uint32_t* qsm;           // this warp's bf16 Q fragments: [kSteps / 2][32 lanes][4]
   Desc* desc;              // this warp's [kEntries] entry descriptions
   uint64_t* bars;          // the CTA's [kEntries] slot barriers
   int* cnt;                // the CTA's [kEntries] counts of warps done with a slot
@@ -126,6 +126,7 @@ struct Worker {
   float kq0, kq1;          // score scale of the thread's score columns: sq * log2(e) * softmax_scale / 64
   float acc[S::kSteps][4];
   float m0, m1, l0, l1, uref, inv_uref;
+  bool q_f16;              // Q of the group fits the f16 range (FP8 pages use f16 products)
 
   __device__ Worker(const DecodeParams& pp, const Prologue& prr, unsigned char* r, uint32_t* q, Desc* d,
                     uint64_t* b, int w)
@@ -261,14 +262,14 @@ struct Worker {
 #pragma unroll
       for (int i = 0; i < S::kWPT * 8; ++i) raw[i] = 0u;
     }
-    // f16 B fragments for FP8 / BF16 pages, kept in shared memory:
-    // fragment ri = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) + (ri & 7)
-    // (thread-local dims), stored at [ri >> 2][lane][ri & 3]
+    // bf16 B fragments for FP8 / BF16 pages (Q as given), kept in shared
+    // memory: fragment ri = (Q[dlo], Q[dlo + 8]), dlo = 16 * (ri >> 3) +
+    // (ri & 7) (thread-local dims), stored at [ri >> 2][lane][ri & 3]
 #pragma unroll
     for (int ri = 0; ri < 2 * S::kSteps; ++ri) {
       const int wl = ri >> 3, j = ri & 7;
       const uint32_t wa = raw[8 * wl + (j >> 1)], wb = raw[8 * wl + 4 + (j >> 1)];
-      const uint32_t v = (NARROW && (gid & 1)) ? 0u : bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
+      const uint32_t v = (NARROW && (gid & 1)) ? 0u : prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u);
       qsm[((ri >> 2) * 32 + lane) * 4 + (ri & 3)] = v;
     }
     // int8 hi/lo B fragments for ternary pages.  Fragment j carries, in
@@ -281,6 +282,7 @@ struct Worker {
     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
     const float inv = amax > 0.f ? 16256.f / amax : 0.f;
+    q_f16 = __all_sync(kFull, amax <= 65504.f);
 #pragma unroll
     for (int j = 0; j < S::kQ8; ++j) {
       uint32_t h = 0u, l = 0u;
@@ -447,7 +449,7 @@ struct Worker {
         const int st = 4 * wl + q4;
         const uint4 qv = qfrag(st >> 1);
         mma16816(t[st & 1], e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16),
-                 (st & 1) ? qv.z : qv.x, (st & 1) ? qv.w : qv.y);
+                 bf16x2_f16((st & 1) ? qv.z : qv.x), bf16x2_f16((st & 1) ? qv.w : qv.y));
       }
     }
 #pragma unroll
@@ -474,9 +476,9 @@ struct Worker {
       for (int q4 = 0; q4 < 4; ++q4) {         // dims j = 2*q4 (+8) and 2*q4+1 (+8)
         const int st = 4 * wl + q4;
         const uint4 qv = qfrag(st >> 1);
-        mma16816(t[st & 1], bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x5410u)),
-                 bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x5410u)), bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x7632u)),
-                 bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)), (st & 1) ? qv.z : qv.x, (st & 1) ? qv.w : qv.y);
+        mma16816_bf16(t[st & 1], prmt(ya[q4], ya[4 + q4], 0x5410u), prmt(yb[q4], yb[4 + q4], 0x5410u),
+                      prmt(ya[q4], ya[4 + q4], 0x7632u), prmt(yb[q4], yb[4 + q4], 0x7632u),
+                      (st & 1) ? qv.z : qv.x, (st & 1) ? qv.w : qv.y);
       }
     }
 #pragma unroll
@@ -571,15 +573,15 @@ struct Worker {
       const int ua = la >> 3, ja = la & 7, ub = lb >> 3, jb = lb & 7;
       const int ba = off + 16 * ua + 4 * (ja >> 1), bb = off + 16 * ub + 4 * (jb >> 1);
       const uint32_t sa = (ja & 1) ? 0x7632u : 0x5410u, sb = (jb & 1) ? 0x7632u : 0x5410u;
-      const uint32_t a0 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + ba), lds<uint32_t>(vg + (t0 + 1) * 2 * D + ba), sa)) & m01;
-      const uint32_t a1 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + bb), lds<uint32_t>(vg + (t0 + 1) * 2 * D + bb), sb)) & m01;
+      const uint32_t a0 = prmt(lds<uint32_t>(vg + t0 * 2 * D + ba), lds<uint32_t>(vg + (t0 + 1) * 2 * D + ba), sa) & m01;
+      const uint32_t a1 = prmt(lds<uint32_t>(vg + t0 * 2 * D + bb), lds<uint32_t>(vg + (t0 + 1) * 2 * D + bb), sb) & m01;
       uint32_t a2 = 0u, a3 = 0u;
       if constexpr (ROWS == 16) {
-        a2 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa)) & m23;
-        a3 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb)) & m23;
+        a2 = prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa) & m23;
+        a3 = prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb) & m23;
       }
-      mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
-      if constexpr (!NARROW) mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
+      mma16816_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
+      if constexpr (!NARROW) mma16816_bf16(acc[mt], a0, a1, a2, a3, lo0, lo1);
     }
   }
 
@@ -593,7 +595,8 @@ struct Worker {
   // NARROW: one query head (tig) per thread, scores s[0] (token gid) and
   // s[2] (token gid + 8) scaled by sc0; P always goes out as the hi + lo pair
   // in columns (2 * tig, 2 * tig + 1), so SPLIT does not apply.
-  template <bool SPLIT>
+  // BF: P goes out in bf16 (BF16 pages multiply V as stored) instead of f16.
+  template <bool SPLIT, bool BF = false>
   // sc0 / sc1 scale the thread's two score columns (s[0], s[2] and s[1], s[3]).
   __device__ __forceinline__ void softmax_page(float (&s)[4], float sc0, float sc1, float ratio, int nt,
                                                uint32_t& b0, uint32_t& b1, uint32_t& lo0, uint32_t& lo1) {
@@ -625,8 +628,13 @@ struct Worker {
       }
       const float p0 = ex2(e0), p1 = ex2(e1);
       l0 += p0 + p1;
-      b0 = movtrans(split_f16x2(p0 * ratio));
-      b1 = movtrans(split_f16x2(p1 * ratio));
+      if constexpr (BF) {
+        b0 = movtrans(split_bf16x2(p0 * ratio));
+        b1 = movtrans(split_bf16x2(p1 * ratio));
+      } else {
+        b0 = movtrans(split_f16x2(p0 * ratio));
+        b1 = movtrans(split_f16x2(p1 * ratio));
+      }
       return;
     }
     // exponent arguments s*sc - m; the scales are >= 0 (gamma, s or 1, times max|q|)
@@ -670,14 +678,24 @@ struct Worker {
     l1 += p01 + p11;
     // P scaled by the page's V scale (relative to the reference)
     const float y00 = p00 * ratio, y01 = p01 * ratio, y10 = p10 * ratio, y11 = p11 * ratio;
-    const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
-    b0 = movtrans(h0);
-    b1 = movtrans(h1);
-    if constexpr (SPLIT) {
-      const float2 g0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-      const float2 g1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-      lo0 = movtrans(f16x2(y00 - g0.x, y01 - g0.y));
-      lo1 = movtrans(f16x2(y10 - g1.x, y11 - g1.y));
+    if constexpr (BF) {
+      const uint32_t h0 = bf16x2(y00, y01), h1 = bf16x2(y10, y11);
+      b0 = movtrans(h0);
+      b1 = movtrans(h1);
+      const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h0));
+      const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h1));
+      lo0 = movtrans(bf16x2(y00 - g0.x, y01 - g0.y));
+      lo1 = movtrans(bf16x2(y10 - g1.x, y11 - g1.y));
+    } else {
+      const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
+      b0 = movtrans(h0);
+      b1 = movtrans(h1);
+      if constexpr (SPLIT) {
+        const float2 g0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+        const float2 g1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+        lo0 = movtrans(f16x2(y00 - g0.x, y01 - g0.y));
+        lo1 = movtrans(f16x2(y10 - g1.x, y11 - g1.y));
+      }
     }
   }
 
@@ -735,6 +753,7 @@ struct Worker {
       constexpr int GB = HPC * group_bytes(KVC_FMT_FP8_E4M3, D);
       e += wi * group_bytes(KVC_FMT_FP8_E4M3, D);
       rebase_value_scale(d, 1.f);
+      if (!q_f16 && lane == 0) atomicOr(p.err, kErrRange);
       for (int i = 0; i < np; ++i) {
         const int nt = i == np - 1 ? d.nrows : kPage;
         float s[4];
@@ -749,11 +768,11 @@ struct Worker {
       float s[4];
       if constexpr (S::kBf16Rows == 16) {
         qk_bf16<16>(e, s);
-        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, b0, b1, lo0, lo1);
+        softmax_page<true, true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, b0, b1, lo0, lo1);
         pv_bf16<16>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       } else {
         qk_bf16<8>(e, s);
-        softmax_page<true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, b0, b1, lo0, lo1);
+        softmax_page<true, true>(s, p.scale_log2, p.scale_log2, inv_uref, d.nrows, b0, b1, lo0, lo1);
         pv_bf16<8>(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
       }
     }

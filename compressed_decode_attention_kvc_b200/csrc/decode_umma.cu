@@ -255,7 +255,8 @@ struct UWorker {
   MetaA nxa;
   bool nxt_b_pending, nxa_pending;
   // high-precision path state (warp h = KV head h)
-  uint32_t qf[2 * S::kSteps];   // f16 Q B-fragments
+  uint32_t qf[2 * S::kSteps];   // bf16 Q B-fragments (Q as given)
+  bool q_f16;                   // Q of the group fits the f16 range (FP8 pages use f16 products)
   float acc[S::kSteps][4];
   float m0, m1, l0, l1, huref, inv_huref;
   int hp_used;
@@ -457,8 +458,13 @@ struct UWorker {
       for (int ri = 0; ri < 2 * S::kSteps; ++ri) {
         const int wl = ri >> 3, j = ri & 7;
         const uint32_t wa = raw[8 * wl + (j >> 1)], wb = raw[8 * wl + 4 + (j >> 1)];
-        qf[ri] = (NARROW && (gid & 1)) ? 0u : bf16x2_f16(prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u));
+        qf[ri] = (NARROW && (gid & 1)) ? 0u : prmt(wa, wb, (j & 1) ? 0x7632u : 0x5410u);
       }
+      float qmax = 0.f;
+#pragma unroll
+      for (int i = 0; i < S::kWPT * 8; ++i)
+        qmax = fmaxf(qmax, fmaxf(fabsf(__uint_as_float(raw[i] << 16)), fabsf(__uint_as_float(raw[i] & 0xFFFF0000u))));
+      q_f16 = __all_sync(kFull, qmax <= 65504.f);
 #pragma unroll
       for (int mt = 0; mt < S::kSteps; ++mt)
 #pragma unroll
@@ -867,8 +873,8 @@ struct UWorker {
         const uint32_t pa = prmt(jj < 4 ? xa.x : xa.y, jj < 4 ? xa.z : xa.w, sel);
         const uint32_t pb = prmt(jj < 4 ? xb.x : xb.y, jj < 4 ? xb.z : xb.w, sel);
         const int st = 4 * wl + q4;
-        mma16816(t[st & 1], e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16), qf[2 * st],
-                 qf[2 * st + 1]);
+        mma16816(t[st & 1], e4m3x2_f16(pa), e4m3x2_f16(pb), e4m3x2_f16(pa >> 16), e4m3x2_f16(pb >> 16),
+                 bf16x2_f16(qf[2 * st]), bf16x2_f16(qf[2 * st + 1]));
       }
     }
 #pragma unroll
@@ -888,9 +894,8 @@ struct UWorker {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const int st = 4 * wl + q4;
-        mma16816(t[st & 1], bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x5410u)), bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x5410u)),
-                 bf16x2_f16(prmt(ya[q4], ya[4 + q4], 0x7632u)), bf16x2_f16(prmt(yb[q4], yb[4 + q4], 0x7632u)),
-                 qf[2 * st], qf[2 * st + 1]);
+        mma16816_bf16(t[st & 1], prmt(ya[q4], ya[4 + q4], 0x5410u), prmt(yb[q4], yb[4 + q4], 0x5410u),
+                      prmt(ya[q4], ya[4 + q4], 0x7632u), prmt(yb[q4], yb[4 + q4], 0x7632u), qf[2 * st], qf[2 * st + 1]);
       }
     }
 #pragma unroll
@@ -941,12 +946,12 @@ struct UWorker {
       const int ua = la >> 3, ja = la & 7, ub = lb >> 3, jb = lb & 7;
       const int ba = off + 16 * ua + 4 * (ja >> 1), bb = off + 16 * ub + 4 * (jb >> 1);
       const uint32_t sa = (ja & 1) ? 0x7632u : 0x5410u, sb = (jb & 1) ? 0x7632u : 0x5410u;
-      const uint32_t a0 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + ba), lds<uint32_t>(vg + (t0 + 1) * 2 * D + ba), sa)) & m01;
-      const uint32_t a1 = bf16x2_f16(prmt(lds<uint32_t>(vg + t0 * 2 * D + bb), lds<uint32_t>(vg + (t0 + 1) * 2 * D + bb), sb)) & m01;
-      const uint32_t a2 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa)) & m23;
-      const uint32_t a3 = bf16x2_f16(prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb)) & m23;
-      mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
-      if constexpr (!NARROW) mma16816(acc[mt], a0, a1, a2, a3, lo0, lo1);
+      const uint32_t a0 = prmt(lds<uint32_t>(vg + t0 * 2 * D + ba), lds<uint32_t>(vg + (t0 + 1) * 2 * D + ba), sa) & m01;
+      const uint32_t a1 = prmt(lds<uint32_t>(vg + t0 * 2 * D + bb), lds<uint32_t>(vg + (t0 + 1) * 2 * D + bb), sb) & m01;
+      const uint32_t a2 = prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + ba), lds<uint32_t>(vg + (t0 + 9) * 2 * D + ba), sa) & m23;
+      const uint32_t a3 = prmt(lds<uint32_t>(vg + (t0 + 8) * 2 * D + bb), lds<uint32_t>(vg + (t0 + 9) * 2 * D + bb), sb) & m23;
+      mma16816_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
+      if constexpr (!NARROW) mma16816_bf16(acc[mt], a0, a1, a2, a3, lo0, lo1);
     }
   }
 
@@ -955,6 +960,8 @@ struct UWorker {
   // the page's V scale relative to the warp's reference), P as an f16 hi + lo
   // pair (~22 bits).  NARROW: one query head (tig) per thread, scores s[0]
   // (token gid) and s[2] (token gid + 8); hi and lo in columns 2 tig, 2 tig + 1.
+  // BF: P goes out in bf16 (BF16 pages multiply V as stored) instead of f16.
+  template <bool BF>
   __device__ __forceinline__ void softmax_page(float (&s)[4], float sc, float ratio, int nt, uint32_t& b0,
                                                uint32_t& b1, uint32_t& lo0, uint32_t& lo1) {
     if constexpr (NARROW) {
@@ -985,8 +992,13 @@ struct UWorker {
       }
       const float p0 = ex2(e0), p1 = ex2(e1);
       l0 += p0 + p1;
-      b0 = movtrans(split_f16x2(p0 * ratio));
-      b1 = movtrans(split_f16x2(p1 * ratio));
+      if constexpr (BF) {
+        b0 = movtrans(split_bf16x2(p0 * ratio));
+        b1 = movtrans(split_bf16x2(p1 * ratio));
+      } else {
+        b0 = movtrans(split_f16x2(p0 * ratio));
+        b1 = movtrans(split_f16x2(p1 * ratio));
+      }
       return;
     }
     float mx0 = fmaxf(s[0], s[2]) * sc, mx1 = fmaxf(s[1], s[3]) * sc;
@@ -1028,13 +1040,23 @@ struct UWorker {
     l0 += p00 + p10;
     l1 += p01 + p11;
     const float y00 = p00 * ratio, y01 = p01 * ratio, y10 = p10 * ratio, y11 = p11 * ratio;
-    const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
-    b0 = movtrans(h0);
-    b1 = movtrans(h1);
-    const float2 g0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-    const float2 g1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-    lo0 = movtrans(f16x2(y00 - g0.x, y01 - g0.y));
-    lo1 = movtrans(f16x2(y10 - g1.x, y11 - g1.y));
+    if constexpr (BF) {
+      const uint32_t h0 = bf16x2(y00, y01), h1 = bf16x2(y10, y11);
+      b0 = movtrans(h0);
+      b1 = movtrans(h1);
+      const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h0));
+      const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h1));
+      lo0 = movtrans(bf16x2(y00 - g0.x, y01 - g0.y));
+      lo1 = movtrans(bf16x2(y10 - g1.x, y11 - g1.y));
+    } else {
+      const uint32_t h0 = f16x2(y00, y01), h1 = f16x2(y10, y11);
+      b0 = movtrans(h0);
+      b1 = movtrans(h1);
+      const float2 g0 = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+      const float2 g1 = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+      lo0 = movtrans(f16x2(y00 - g0.x, y01 - g0.y));
+      lo1 = movtrans(f16x2(y10 - g1.x, y11 - g1.y));
+    }
   }
 
   // Re-base the warp's value-scale reference when the entry's V scales leave
@@ -1064,20 +1086,21 @@ struct UWorker {
     rebase_value_scale(d);
     hp_used = 1;
     if (d.fmt == KVC_FMT_FP8_E4M3) {
+      if (!q_f16 && lane == 0) atomicOr(p.err, kErrRange);
       constexpr int GB = HPC * group_bytes(KVC_FMT_FP8_E4M3, D);
       e += warp * group_bytes(KVC_FMT_FP8_E4M3, D);
       for (int i = 0; i < d.np; ++i) {
         const int nt = i == d.np - 1 ? d.nrows : kPage;
         float s[4];
         qk_fp8(e + i * GB, s);
-        softmax_page(s, d.ks[i] * p.scale_log2, d.vs[i] * inv_huref, nt, b0, b1, lo0, lo1);
+        softmax_page<false>(s, d.ks[i] * p.scale_log2, d.vs[i] * inv_huref, nt, b0, b1, lo0, lo1);
         pv_fp8(e + S::kHalf + i * GB, b0, b1, lo0, lo1, nt);
       }
     } else {
       e += warp * group_bytes(KVC_FMT_BF16, D);
       float s[4];
       qk_bf16(e, s);
-      softmax_page(s, p.scale_log2, inv_huref, d.nrows, b0, b1, lo0, lo1);
+      softmax_page<true>(s, p.scale_log2, inv_huref, d.nrows, b0, b1, lo0, lo1);
       pv_bf16(e + S::kHalf, b0, b1, lo0, lo1, d.nrows);
     }
   }

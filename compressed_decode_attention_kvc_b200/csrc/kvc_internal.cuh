@@ -18,6 +18,7 @@ constexpr uint32_t kErrBlockTable = 1u;
 constexpr uint32_t kErrFormat = 2u;
 constexpr uint32_t kErrContext = 4u;
 constexpr uint32_t kErrTimeout = 8u;
+constexpr uint32_t kErrRange = 16u;   // a query value outside the f16 range met an FP8 page
 
 // Format of logical page j (length-L sequence): the high-precision format
 // if the page holds any of the first `sink` tokens or any of the last

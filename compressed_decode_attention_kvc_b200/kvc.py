@@ -38,6 +38,7 @@ ERR_BLOCK_TABLE = 1
 ERR_FORMAT = 2
 ERR_CONTEXT = 4
 ERR_TIMEOUT = 8
+ERR_RANGE = 16
 
 EXPORTS = (
     "kvc_status_string", "kvc_quantize_pack_pages", "kvc_dequantize_pages",

@@ -434,7 +434,10 @@ KVC_API kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const k
  * kvc_decode_read_error - synchronise `stream`, then read and clear the
  * device error flags in `workspace` (as sized for these shapes).  *flags
  * receives a bit mask: 1 = block-table entry out of range, 2 = unknown page
- * format, 4 = context length out of range, 8 = a bounded wait timed out.
+ * format, 4 = context length out of range, 8 = a bounded wait timed out,
+ * 16 = a query value beyond the f16 range (|q| > 65504) met an FP8 page, whose
+ * products are taken in f16 (its output rows are then not reliable; BF16
+ * and ternary pages take any finite bf16 Q, K and V).
  * Returns KVC_OK, or KVC_ERR_CUDA if the copy failed.
  */
 KVC_API kvc_status kvc_decode_read_error(void* workspace, int batch, int n_q_heads, int n_kv_heads,
