@@ -78,6 +78,7 @@ struct EncSmem {
 // backwards from its end, then moved down behind the escapes.
 __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint16_t* __restrict__ src,
                                                                     const int32_t* __restrict__ page_ids,
+                                                                    long long n_src, uint32_t* flags,
                                                                     int n, long long N, unsigned char* ws) {
   __shared__ EncSmem smem[kExWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,7 +86,11 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint1
   if (g >= n) return;
   EncSmem& S = smem[warp];
   const unsigned lt = lanemask_lt();
-  const long long pid = page_ids ? (long long)page_ids[g] : g;
+  long long pid = page_ids ? (long long)__ldg(page_ids + g) : g;
+  if (pid < 0 || pid >= n_src) {          // an id outside the source: code page 0, flag it
+    if (flags && lane == 0) atomicOr(flags, 1u);
+    pid = 0;
+  }
   const uint16_t* x = src + pid * N;
   const long long cap = 4 * N + 192;
   unsigned char* slot = ws + g * cap;
@@ -465,11 +470,11 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_decode_kernel(const unsig
 
 long long exans_slot_bytes(long long group_elems) { return 4 * group_elems + 192; }
 
-cudaError_t launch_exans_encode(const void* src, const int32_t* page_ids, int n, long long group_elems,
-                                void* ws, long long* offsets, void* dst, cudaStream_t s) {
+cudaError_t launch_exans_encode(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n,
+                                long long group_elems, void* ws, long long* offsets, void* dst, cudaStream_t s) {
   const int grid = (int)((n + kExWarps - 1) / kExWarps);
   auto* w = static_cast<unsigned char*>(ws);
-  exans_encode_kernel<<<grid, kExWarps * 32, 0, s>>>(static_cast<const uint16_t*>(src), page_ids, n,
+  exans_encode_kernel<<<grid, kExWarps * 32, 0, s>>>(static_cast<const uint16_t*>(src), page_ids, n_src, flags, n,
                                                      group_elems, w);
   const long long cap = exans_slot_bytes(group_elems);
   exans_scan_kernel<<<1, 1024, 0, s>>>(w, cap, n, offsets);

@@ -128,34 +128,42 @@ int kvc_layout_version(void) { return KVC_LAYOUT_VERSION; }
 
 kvc_status kvc_quantize_pack_pages(const void* src_bf16, const int32_t* page_ids, int n,
                                    int page_size, int n_kv_heads, int head_dim, kvc_format mode,
-                                   void* dst, float* dst_scale, kvc_stream_t stream) {
+                                   void* dst, float* dst_scale, int64_t n_src_pages,
+                                   uint32_t* device_flags, kvc_stream_t stream) {
   kvc_status st = check_codec(src_bf16, dst, n, page_size, n_kv_heads, head_dim, mode, dst_scale);
   if (st != KVC_OK || n == 0) return st;
+  if (n_src_pages < 1 || (!page_ids && n_src_pages < n)) return KVC_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (mode) {
     case KVC_FMT_TERNARY2:
-      return from_cuda(kvc::launch_quant_ternary(src_bf16, page_ids, n, n_kv_heads, head_dim, dst, dst_scale, s));
+      return from_cuda(kvc::launch_quant_ternary(src_bf16, page_ids, n_src_pages, device_flags, n, n_kv_heads,
+                                                 head_dim, dst, dst_scale, s));
     case KVC_FMT_FP8_E4M3:
-      return from_cuda(kvc::launch_quant_fp8(src_bf16, page_ids, n, n_kv_heads, head_dim, dst, dst_scale, s));
+      return from_cuda(kvc::launch_quant_fp8(src_bf16, page_ids, n_src_pages, device_flags, n, n_kv_heads, head_dim,
+                                             dst, dst_scale, s));
     default:
-      return from_cuda(kvc::launch_copy_pages(src_bf16, page_ids, n,
+      return from_cuda(kvc::launch_copy_pages(src_bf16, page_ids, n_src_pages, device_flags, n,
                                               (size_t)n_kv_heads * KVC_PAGE_SIZE * head_dim * 2, dst, s));
   }
 }
 
 kvc_status kvc_dequantize_pages(const void* src, const float* src_scale, const int32_t* page_ids,
                                 int n, int page_size, int n_kv_heads, int head_dim,
-                                kvc_format mode, void* dst_bf16, kvc_stream_t stream) {
+                                kvc_format mode, void* dst_bf16, int64_t n_src_pages, uint32_t* device_flags,
+                                kvc_stream_t stream) {
   kvc_status st = check_codec(src, dst_bf16, n, page_size, n_kv_heads, head_dim, mode, src_scale);
   if (st != KVC_OK || n == 0) return st;
+  if (n_src_pages < 1 || (!page_ids && n_src_pages < n)) return KVC_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (mode) {
     case KVC_FMT_TERNARY2:
-      return from_cuda(kvc::launch_dequant_ternary(src, src_scale, page_ids, n, n_kv_heads, head_dim, dst_bf16, s));
+      return from_cuda(kvc::launch_dequant_ternary(src, src_scale, page_ids, n_src_pages, device_flags, n, n_kv_heads,
+                                                   head_dim, dst_bf16, s));
     case KVC_FMT_FP8_E4M3:
-      return from_cuda(kvc::launch_dequant_fp8(src, src_scale, page_ids, n, n_kv_heads, head_dim, dst_bf16, s));
+      return from_cuda(kvc::launch_dequant_fp8(src, src_scale, page_ids, n_src_pages, device_flags, n, n_kv_heads,
+                                               head_dim, dst_bf16, s));
     default:
-      return from_cuda(kvc::launch_copy_pages(src, page_ids, n,
+      return from_cuda(kvc::launch_copy_pages(src, page_ids, n_src_pages, device_flags, n,
                                               (size_t)n_kv_heads * KVC_PAGE_SIZE * head_dim * 2, dst_bf16, s));
   }
 }
@@ -242,7 +250,8 @@ kvc_status kvc_exans_workspace_size(int n, int page_size, int n_kv_heads, int he
 
 kvc_status kvc_exans_encode(const void* src_bf16, const int32_t* page_ids, int n, int page_size,
                             int n_kv_heads, int head_dim, void* workspace, size_t workspace_bytes, void* dst,
-                            size_t dst_bytes, int64_t* offsets, kvc_stream_t stream) {
+                            size_t dst_bytes, int64_t* offsets, int64_t n_src_pages, uint32_t* device_flags,
+                            kvc_stream_t stream) {
   if (n < 0 || n > (1 << 24)) return KVC_ERR_INVALID_ARG;
   const long long N = exans_group_elems(page_size, n_kv_heads, head_dim);
   if (N < 0) return KVC_ERR_UNSUPPORTED;
@@ -253,7 +262,8 @@ kvc_status kvc_exans_encode(const void* src_bf16, const int32_t* page_ids, int n
   if (!workspace || !aligned(workspace, 16) || workspace_bytes < (size_t)n * (size_t)kvc::exans_slot_bytes(N))
     return KVC_ERR_WORKSPACE;
   if (dst_bytes < (size_t)n * (size_t)(64 + 2 * N)) return KVC_ERR_INVALID_ARG;
-  return from_cuda(kvc::launch_exans_encode(src_bf16, page_ids, n, N, workspace,
+  if (n_src_pages < 1 || (!page_ids && n_src_pages < n)) return KVC_ERR_INVALID_ARG;
+  return from_cuda(kvc::launch_exans_encode(src_bf16, page_ids, n_src_pages, device_flags, n, N, workspace,
                                             reinterpret_cast<long long*>(offsets), dst,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -370,8 +380,11 @@ kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged
   if (batch == 0) return KVC_OK;
   if (!q_bf16 || !cache || !block_table || !context_lens || !out) return KVC_ERR_INVALID_ARG;
   if (!aligned(q_bf16, 16) || !aligned(out, 16)) return KVC_ERR_INVALID_ARG;
-  for (int f = 0; f < 3; ++f)
+  for (int f = 0; f < 3; ++f) {
     if (cache->n_pages[f] < 0) return KVC_ERR_INVALID_ARG;
+    // group indices (layer * n_pages + slot) * Hkv + head are 32-bit in the kernels
+    if ((long long)n_layers * cache->n_pages[f] * n_kv_heads >= (1ll << 31)) return KVC_ERR_UNSUPPORTED;
+  }
   if (cache->n_pages[KVC_FMT_BF16] > 0 &&
       (!cache->k_bf16 || !cache->v_bf16 || !aligned(cache->k_bf16, 16) || !aligned(cache->v_bf16, 16)))
     return KVC_ERR_INVALID_ARG;
@@ -388,6 +401,10 @@ kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged
   if (kvc::decode_plan(batch, n_q_heads, n_kv_heads, head_dim, max_pages, &plan) != cudaSuccess)
     return KVC_ERR_CUDA;
   if (!workspace || workspace_bytes < plan.bytes || !aligned(workspace, 256)) return KVC_ERR_WORKSPACE;
+  // error word and merge tickets start at zero on every call, so a call that
+  // gave up on a wait (and left tickets behind) cannot poison the next one
+  if (cudaMemsetAsync(workspace, 0, plan.partial_offset, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KVC_ERR_CUDA;
 
   kvc::DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q_bf16);

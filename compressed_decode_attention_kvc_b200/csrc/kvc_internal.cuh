@@ -32,21 +32,24 @@ __host__ __device__ __forceinline__ int page_format(int j, int L, int sink, int 
 }
 
 // ---------------------------------------------------------------- quantise
-cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, int n, int hkv, int d,
-                                 void* dst, float* gamma, cudaStream_t s);
-cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, int n, int hkv, int d,
-                             void* dst, float* scale, cudaStream_t s);
-cudaError_t launch_copy_pages(const void* src, const int32_t* page_ids, int n,
+// page_ids[i] (or i when page_ids is NULL) names the source page of output
+// page i; ids outside [0, n_src) skip that output page and set bit 1 of
+// *flags (when flags is not NULL).
+cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n,
+                                 int hkv, int d, void* dst, float* gamma, cudaStream_t s);
+cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n,
+                             int hkv, int d, void* dst, float* scale, cudaStream_t s);
+cudaError_t launch_copy_pages(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n,
                               size_t page_bytes, void* dst, cudaStream_t s);
-cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const int32_t* page_ids,
-                                   int n, int hkv, int d, void* dst, cudaStream_t s);
-cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids,
-                               int n, int hkv, int d, void* dst, cudaStream_t s);
+cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const int32_t* page_ids, long long n_src,
+                                   uint32_t* flags, int n, int hkv, int d, void* dst, cudaStream_t s);
+cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids, long long n_src,
+                               uint32_t* flags, int n, int hkv, int d, void* dst, cudaStream_t s);
 
 // exponent-split lossless codec of BF16 pages (exans.cu)
 long long exans_slot_bytes(long long group_elems);
-cudaError_t launch_exans_encode(const void* src, const int32_t* page_ids, int n, long long group_elems,
-                                void* ws, long long* offsets, void* dst, cudaStream_t s);
+cudaError_t launch_exans_encode(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n,
+                                long long group_elems, void* ws, long long* offsets, void* dst, cudaStream_t s);
 cudaError_t launch_exans_decode(const void* src, long long src_bytes, const long long* offsets, int n_blobs,
                                 const int32_t* ids, int n, long long group_elems, void* dst, uint32_t* flags,
                                 cudaStream_t s);

@@ -68,14 +68,9 @@ kvc_status kvc_decode_attention_paged_noalloc(const void* q_bf16, const kvc_page
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != KVC_OK) return st;
-  // The scratch keeps whatever the previous call left: clear the error word
-  // and the merge tickets, which must start at zero.
-  kvc::DecodePlan plan;
-  if (kvc::decode_plan(batch, n_q_heads, n_kv_heads, head_dim, max_pages, &plan) != cudaSuccess)
-    return KVC_ERR_CUDA;
-  if (cudaMemsetAsync(scratch, 0, plan.partial_offset, reinterpret_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
-    return KVC_ERR_CUDA;
+  // The scratch keeps whatever the previous call left; the regular entry
+  // point clears the error word and the merge tickets on every call (one
+  // cudaMemsetAsync on `stream`) and rewrites the partial states.
   return kvc_decode_attention_paged(q_bf16, cache, block_table, older_fmt, context_lens, batch,
                                     n_q_heads, n_kv_heads, head_dim, page_size, max_pages,
                                     sink_tokens, window_tokens, hp_mode, softmax_scale, out,

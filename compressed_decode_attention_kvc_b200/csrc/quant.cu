@@ -61,9 +61,22 @@ __device__ __forceinline__ uint32_t tern_word16(const uint4& v, float t) {
 // of the warp is contiguous.  gamma is a pairwise tree (per chunk, across the
 // lane's chunks, across lanes, across the parts): depth log2(16*D) <= 12, so
 // its float32 relative error stays below 12 * 2^-24.
+// Source page of output page i, or -1 when page_ids[i] lies outside
+// [0, n_src): the caller skips that output page and flag 1 is raised.
+__device__ __forceinline__ long long src_page(const int32_t* __restrict__ ids, long long i, long long n_src,
+                                              uint32_t* flags) {
+  const long long sp = ids ? (long long)__ldg(ids + i) : i;
+  if (sp < 0 || sp >= n_src) {
+    if (flags) atomicOr(flags, 1u);
+    return -1;
+  }
+  return sp;
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) quant_ternary_kernel(const uint4* __restrict__ src,
                                                             const int32_t* __restrict__ page_ids,
+                                                            long long n_src, uint32_t* flags,
                                                             long long n_groups, int hkv,
                                                             uint16_t* __restrict__ dst,
                                                             float* __restrict__ gamma) {
@@ -73,12 +86,13 @@ __global__ void __launch_bounds__(256) quant_ternary_kernel(const uint4* __restr
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int part = warp % WPG;
   const long long grp = (long long)blockIdx.x * (8 / WPG) + warp / WPG;
-  const bool valid = grp < n_groups;
+  bool valid = grp < n_groups;
   const uint4* s = src;
   if (valid) {
     const long long i = grp / hkv;
     const int h = (int)(grp - i * hkv);
-    const long long sp = page_ids ? (long long)page_ids[i] : i;
+    const long long sp = src_page(page_ids, i, n_src, flags);
+    valid = sp >= 0;
     s = src + (sp * hkv + h) * (2 * D) + part * (NC * 32);
   }
 
@@ -119,12 +133,14 @@ __global__ void __launch_bounds__(256) quant_ternary_kernel(const uint4* __restr
 // page from L2 (a page is at most a few hundred KB), so DRAM sees it once.
 __global__ void __launch_bounds__(256) quant_fp8_kernel(const uint4* __restrict__ src,
                                                         const int32_t* __restrict__ page_ids,
+                                                        long long n_src, uint32_t* flags,
                                                         int chunks_per_page,
                                                         uint2* __restrict__ dst,
                                                         float* __restrict__ scale) {
   __shared__ float red[8];
   const long long i = blockIdx.x;
-  const long long sp = page_ids ? (long long)page_ids[i] : i;
+  const long long sp = src_page(page_ids, i, n_src, flags);
+  if (sp < 0) return;                       // uniform over the CTA
   const uint4* s = src + sp * chunks_per_page;
   float amax = 0.f;
   for (int c = threadIdx.x; c < chunks_per_page; c += 256) {
@@ -167,18 +183,20 @@ __global__ void __launch_bounds__(256) quant_fp8_kernel(const uint4* __restrict_
 // the encode is the same float32 arithmetic as quant_fp8_kernel.
 template <int WPP, int CPL>
 __global__ void __launch_bounds__(256, 3) quant_fp8_reg_kernel(const uint4* __restrict__ src,
-                                                            const int32_t* __restrict__ page_ids, int n,
+                                                            const int32_t* __restrict__ page_ids,
+                                                            long long n_src, uint32_t* flags, int n,
                                                             uint2* __restrict__ dst, float* __restrict__ scale) {
   constexpr int CPP = WPP * 32 * CPL;        // chunks per page
   __shared__ float red[8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int part = warp % WPP;
   const long long i = (long long)blockIdx.x * (8 / WPP) + warp / WPP;
-  const bool valid = i < n;
+  bool valid = i < n;
   uint4 v[CPL];
   float amax = 0.f;
+  const long long sp = valid ? src_page(page_ids, i, n_src, flags) : -1;
+  valid = sp >= 0;
   if (valid) {
-    const long long sp = page_ids ? (long long)page_ids[i] : i;
     const uint4* s = src + sp * CPP + part * (32 * CPL);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) v[c] = ld_stream(s + c * 32 + lane);
@@ -220,13 +238,14 @@ __global__ void __launch_bounds__(256, 3) quant_fp8_reg_kernel(const uint4* __re
 
 __global__ void __launch_bounds__(256) copy_pages_kernel(const uint4* __restrict__ src,
                                                          const int32_t* __restrict__ page_ids,
+                                                         long long n_src, uint32_t* flags,
                                                          long long n_chunks, long long cpp,
                                                          uint4* __restrict__ dst) {
   for (long long c = (long long)blockIdx.x * 256 + threadIdx.x; c < n_chunks;
        c += (long long)gridDim.x * 256) {
     const long long i = c / cpp;
-    const long long sp = page_ids ? (long long)page_ids[i] : i;
-    dst[c] = ld_stream(src + sp * cpp + (c - i * cpp));
+    const long long sp = src_page(page_ids, i, n_src, flags);
+    if (sp >= 0) dst[c] = ld_stream(src + sp * cpp + (c - i * cpp));
   }
 }
 
@@ -236,6 +255,7 @@ template <int D>
 __global__ void __launch_bounds__(256) dequant_ternary_kernel(const uint16_t* __restrict__ src,
                                                               const float* __restrict__ gamma,
                                                               const int32_t* __restrict__ page_ids,
+                                                              long long n_src, uint32_t* flags,
                                                               long long n_groups, int hkv,
                                                               uint4* __restrict__ dst) {
   constexpr int NC = D / 16;
@@ -244,7 +264,9 @@ __global__ void __launch_bounds__(256) dequant_ternary_kernel(const uint16_t* __
   if (grp >= n_groups) return;
   const long long i = grp / hkv;
   const int h = (int)(grp - i * hkv);
-  const long long sg = (page_ids ? (long long)page_ids[i] : i) * hkv + h;
+  const long long sp = src_page(page_ids, i, n_src, flags);
+  if (sp < 0) return;
+  const long long sg = sp * hkv + h;
   const uint16_t* s = src + sg * (2 * D);
   const uint32_t pos = __bfloat16_as_ushort(__float2bfloat16_rn(__ldg(gamma + sg)));
   const uint32_t neg = pos | 0x8000u;
@@ -270,12 +292,14 @@ __global__ void __launch_bounds__(256) dequant_ternary_kernel(const uint16_t* __
 __global__ void __launch_bounds__(256) dequant_fp8_kernel(const uint2* __restrict__ src,
                                                           const float* __restrict__ scale,
                                                           const int32_t* __restrict__ page_ids,
+                                                          long long n_src, uint32_t* flags,
                                                           long long n_chunks, long long cpp,
                                                           uint4* __restrict__ dst) {
   for (long long c = (long long)blockIdx.x * 256 + threadIdx.x; c < n_chunks;
        c += (long long)gridDim.x * 256) {
     const long long i = c / cpp;
-    const long long sp = page_ids ? (long long)page_ids[i] : i;
+    const long long sp = src_page(page_ids, i, n_src, flags);
+    if (sp < 0) continue;
     const float s = __ldg(scale + sp);
     const uint2 e = __ldg(src + sp * cpp + (c - i * cpp));
     const uint32_t ew[2] = {e.x, e.y};
@@ -661,22 +685,22 @@ int grid_for(long long work, int per_block) {
 
 }  // namespace
 
-cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, int n, int hkv, int d,
+cudaError_t launch_quant_ternary(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n, int hkv, int d,
                                  void* dst, float* gamma, cudaStream_t s) {
   const long long groups = (long long)n * hkv;
   const int grid = grid_for(groups, d > 128 ? 2 : 8);      // groups per 256-thread CTA
   auto* in = static_cast<const uint4*>(src);
   auto* out = static_cast<uint16_t*>(dst);
   switch (d) {
-    case 64: quant_ternary_kernel<64><<<grid, 256, 0, s>>>(in, page_ids, groups, hkv, out, gamma); break;
-    case 128: quant_ternary_kernel<128><<<grid, 256, 0, s>>>(in, page_ids, groups, hkv, out, gamma); break;
-    case 256: quant_ternary_kernel<256><<<grid, 256, 0, s>>>(in, page_ids, groups, hkv, out, gamma); break;
+    case 64: quant_ternary_kernel<64><<<grid, 256, 0, s>>>(in, page_ids, n_src, flags, groups, hkv, out, gamma); break;
+    case 128: quant_ternary_kernel<128><<<grid, 256, 0, s>>>(in, page_ids, n_src, flags, groups, hkv, out, gamma); break;
+    case 256: quant_ternary_kernel<256><<<grid, 256, 0, s>>>(in, page_ids, n_src, flags, groups, hkv, out, gamma); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, int n, int hkv, int d,
+cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n, int hkv, int d,
                              void* dst, float* scale, cudaStream_t s) {
   const int cpp = hkv * kPage * d / 8;
   auto* in = static_cast<const uint4*>(src);
@@ -686,34 +710,34 @@ cudaError_t launch_quant_fp8(const void* src, const int32_t* page_ids, int n, in
   switch (cpp) {
     // (measured: 4 warps x 4 chunks per lane for 8 KB pages and 8 x 8 for
     // 32 KB pages beat 2 x 8 / 8 x 2 and 4 x 16)
-    case 512: quant_fp8_reg_kernel<4, 4><<<grid_for(n, 2), 256, 0, s>>>(in, page_ids, n, out, scale); break;
-    case 1024: quant_fp8_reg_kernel<4, 8><<<grid_for(n, 2), 256, 0, s>>>(in, page_ids, n, out, scale); break;
-    case 2048: quant_fp8_reg_kernel<8, 8><<<n, 256, 0, s>>>(in, page_ids, n, out, scale); break;
-    case 4096: quant_fp8_reg_kernel<8, 16><<<n, 256, 0, s>>>(in, page_ids, n, out, scale); break;
-    default: quant_fp8_kernel<<<n, 256, 0, s>>>(in, page_ids, cpp, out, scale); break;
+    case 512: quant_fp8_reg_kernel<4, 4><<<grid_for(n, 2), 256, 0, s>>>(in, page_ids, n_src, flags, n, out, scale); break;
+    case 1024: quant_fp8_reg_kernel<4, 8><<<grid_for(n, 2), 256, 0, s>>>(in, page_ids, n_src, flags, n, out, scale); break;
+    case 2048: quant_fp8_reg_kernel<8, 8><<<n, 256, 0, s>>>(in, page_ids, n_src, flags, n, out, scale); break;
+    case 4096: quant_fp8_reg_kernel<8, 16><<<n, 256, 0, s>>>(in, page_ids, n_src, flags, n, out, scale); break;
+    default: quant_fp8_kernel<<<n, 256, 0, s>>>(in, page_ids, n_src, flags, cpp, out, scale); break;
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_copy_pages(const void* src, const int32_t* page_ids, int n, size_t page_bytes,
+cudaError_t launch_copy_pages(const void* src, const int32_t* page_ids, long long n_src, uint32_t* flags, int n, size_t page_bytes,
                               void* dst, cudaStream_t s) {
   const long long cpp = (long long)(page_bytes / 16);
   const long long chunks = cpp * n;
   copy_pages_kernel<<<grid_for(chunks, 256 * 4), 256, 0, s>>>(
-      static_cast<const uint4*>(src), page_ids, chunks, cpp, static_cast<uint4*>(dst));
+      static_cast<const uint4*>(src), page_ids, n_src, flags, chunks, cpp, static_cast<uint4*>(dst));
   return cudaGetLastError();
 }
 
-cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const int32_t* page_ids,
+cudaError_t launch_dequant_ternary(const void* src, const float* gamma, const int32_t* page_ids, long long n_src, uint32_t* flags,
                                    int n, int hkv, int d, void* dst, cudaStream_t s) {
   const long long groups = (long long)n * hkv;
   const int grid = grid_for(groups, 8);
   auto* in = static_cast<const uint16_t*>(src);
   auto* out = static_cast<uint4*>(dst);
   switch (d) {
-    case 64: dequant_ternary_kernel<64><<<grid, 256, 0, s>>>(in, gamma, page_ids, groups, hkv, out); break;
-    case 128: dequant_ternary_kernel<128><<<grid, 256, 0, s>>>(in, gamma, page_ids, groups, hkv, out); break;
-    case 256: dequant_ternary_kernel<256><<<grid, 256, 0, s>>>(in, gamma, page_ids, groups, hkv, out); break;
+    case 64: dequant_ternary_kernel<64><<<grid, 256, 0, s>>>(in, gamma, page_ids, n_src, flags, groups, hkv, out); break;
+    case 128: dequant_ternary_kernel<128><<<grid, 256, 0, s>>>(in, gamma, page_ids, n_src, flags, groups, hkv, out); break;
+    case 256: dequant_ternary_kernel<256><<<grid, 256, 0, s>>>(in, gamma, page_ids, n_src, flags, groups, hkv, out); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -779,12 +803,12 @@ cudaError_t launch_promote(const kvc_paged_cache& cache, int32_t* block_table, u
   return cudaGetLastError();
 }
 
-cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids,
+cudaError_t launch_dequant_fp8(const void* src, const float* scale, const int32_t* page_ids, long long n_src, uint32_t* flags,
                                int n, int hkv, int d, void* dst, cudaStream_t s) {
   const long long cpp = (long long)hkv * kPage * d / 8;
   const long long chunks = cpp * n;
   dequant_fp8_kernel<<<grid_for(chunks, 256 * 4), 256, 0, s>>>(
-      static_cast<const uint2*>(src), scale, page_ids, chunks, cpp, static_cast<uint4*>(dst));
+      static_cast<const uint2*>(src), scale, page_ids, n_src, flags, chunks, cpp, static_cast<uint4*>(dst));
   return cudaGetLastError();
 }
 

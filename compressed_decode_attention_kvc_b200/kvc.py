@@ -80,9 +80,9 @@ def _load() -> ctypes.CDLL:
     lib.kvc_layout_version.restype = ctypes.c_int
     lib.kvc_layout_version.argtypes = []
     lib.kvc_quantize_pack_pages.restype = st
-    lib.kvc_quantize_pack_pages.argtypes = [vp, vp, i32, i32, i32, i32, st, vp, vp, vp]
+    lib.kvc_quantize_pack_pages.argtypes = [vp, vp, i32, i32, i32, i32, st, vp, vp, ctypes.c_int64, vp, vp]
     lib.kvc_dequantize_pages.restype = st
-    lib.kvc_dequantize_pages.argtypes = [vp, vp, vp, i32, i32, i32, i32, st, vp, vp]
+    lib.kvc_dequantize_pages.argtypes = [vp, vp, vp, i32, i32, i32, i32, st, vp, ctypes.c_int64, vp, vp]
     lib.kvc_append_retier.restype = st
     lib.kvc_append_retier.argtypes = [vp, vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, vp, vp, vp,
                                       i32, i32, i32, i32, i32, i32, i32, st, vp]
@@ -93,7 +93,7 @@ def _load() -> ctypes.CDLL:
     lib.kvc_exans_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.kvc_exans_encode.restype = st
     lib.kvc_exans_encode.argtypes = [vp, vp, i32, i32, i32, i32, vp, ctypes.c_size_t, vp, ctypes.c_size_t, vp,
-                                     vp]
+                                     ctypes.c_int64, vp, vp]
     lib.kvc_exans_decode.restype = st
     lib.kvc_exans_decode.argtypes = [vp, ctypes.c_size_t, vp, i32, vp, i32, i32, i32, i32, vp, vp, vp]
     lib.kvc_plan_paged_cache.restype = st
@@ -147,17 +147,33 @@ def kvc_status_string(status: int) -> str:
     return _lib.kvc_status_string(status).decode()
 
 
+def _src_pages(src, n_src_pages, page_bytes: int, n: int) -> int:
+    """Pages in a source buffer: the caller's count, else the tensor's size
+    divided by the bytes of one page (a raw pointer without a count is taken
+    to hold n pages)."""
+    if n_src_pages is not None:
+        return int(n_src_pages)
+    if isinstance(src, torch.Tensor):
+        return src.numel() * src.element_size() // page_bytes
+    return max(1, int(n))
+
+
 def kvc_quantize_pack_pages(src_bf16, page_ids, n, page_size, n_kv_heads, head_dim, mode,
-                            dst, dst_scale, stream=None) -> None:
+                            dst, dst_scale, stream=None, n_src_pages=None, device_flags=None) -> None:
+    ns = _src_pages(src_bf16, n_src_pages, 2 * page_size * n_kv_heads * head_dim, n) if n else 0
     _check(_lib.kvc_quantize_pack_pages(_ptr(src_bf16), _ptr(page_ids), n, page_size, n_kv_heads,
-                                        head_dim, mode, _ptr(dst), _ptr(dst_scale), _stream(stream)),
+                                        head_dim, mode, _ptr(dst), _ptr(dst_scale), ns, _ptr(device_flags),
+                                        _stream(stream)),
            "kvc_quantize_pack_pages")
 
 
 def kvc_dequantize_pages(src, src_scale, page_ids, n, page_size, n_kv_heads, head_dim, mode,
-                         dst_bf16, stream=None) -> None:
+                         dst_bf16, stream=None, n_src_pages=None, device_flags=None) -> None:
+    per = {KVC_FMT_BF16: 2, KVC_FMT_FP8_E4M3: 1}.get(mode, 0.25)
+    ns = _src_pages(src, n_src_pages, int(per * page_size * n_kv_heads * head_dim), n) if n else 0
     _check(_lib.kvc_dequantize_pages(_ptr(src), _ptr(src_scale), _ptr(page_ids), n, page_size,
-                                     n_kv_heads, head_dim, mode, _ptr(dst_bf16), _stream(stream)),
+                                     n_kv_heads, head_dim, mode, _ptr(dst_bf16), ns, _ptr(device_flags),
+                                     _stream(stream)),
            "kvc_dequantize_pages")
 
 
@@ -201,11 +217,12 @@ def kvc_exans_workspace_size(n, page_size, n_kv_heads, head_dim) -> int:
 
 
 def kvc_exans_encode(src_bf16, page_ids, n, page_size, n_kv_heads, head_dim, workspace, workspace_bytes, dst,
-                     dst_bytes, offsets, stream=None) -> None:
+                     dst_bytes, offsets, stream=None, n_src_pages=None, device_flags=None) -> None:
     """Lossless exponent-split coding of n BF16 pages (see include/kvc.h)."""
+    ns = _src_pages(src_bf16, n_src_pages, 2 * page_size * n_kv_heads * head_dim, n) if n else 0
     _check(_lib.kvc_exans_encode(_ptr(src_bf16), _ptr(page_ids), n, page_size, n_kv_heads, head_dim,
                                  _ptr(workspace), int(workspace_bytes), _ptr(dst), int(dst_bytes), _ptr(offsets),
-                                 _stream(stream)),
+                                 ns, _ptr(device_flags), _stream(stream)),
            "kvc_exans_encode")
 
 

@@ -114,16 +114,21 @@ KVC_API int kvc_layout_version(void);
  *
  *   src_bf16   device, bf16 [n_src][Hkv][16][D]; 16-byte aligned
  *   page_ids   device int32 [n]: dst page i is made from src page
- *              page_ids[i]; NULL means page_ids[i] = i.  Entries must lie in
- *              [0, n_src) (not checked on the device).
+ *              page_ids[i]; NULL means page_ids[i] = i
  *   n          number of pages to produce (0 is a no-op)
  *   page_size  must be 16
  *   dst        device, layout of `mode` [n][...]; 16-byte aligned
  *   dst_scale  device float32, [n][Hkv] (ternary) or [n] (FP8)
+ *   n_src_pages  pages in src (>= 1; >= n when page_ids is NULL)
+ *   device_flags device uint32 or NULL: an id outside [0, n_src_pages) is
+ *              checked on the device, its dst page (and scale) left as it
+ *              was, and bit 1 set in *device_flags (atomicOr; the caller
+ *              zeroes and reads it)
  */
 KVC_API kvc_status kvc_quantize_pack_pages(const void* src_bf16, const int32_t* page_ids, int n,
                                    int page_size, int n_kv_heads, int head_dim,
                                    kvc_format mode, void* dst, float* dst_scale,
+                                   int64_t n_src_pages, uint32_t* device_flags,
                                    kvc_stream_t stream);
 
 /*
@@ -138,10 +143,13 @@ KVC_API kvc_status kvc_quantize_pack_pages(const void* src_bf16, const int32_t* 
  *   page_ids   device int32 [n] or NULL: dst page i is made from src page
  *              page_ids[i] (NULL: i)
  *   dst_bf16   device bf16 [n][Hkv][16][D]; 16-byte aligned
+ *   n_src_pages, device_flags   as for kvc_quantize_pack_pages (an id
+ *              outside the source leaves its dst page as it was, bit 1)
  */
 KVC_API kvc_status kvc_dequantize_pages(const void* src, const float* src_scale, const int32_t* page_ids,
                                 int n, int page_size, int n_kv_heads, int head_dim,
-                                kvc_format mode, void* dst_bf16, kvc_stream_t stream);
+                                kvc_format mode, void* dst_bf16, int64_t n_src_pages,
+                                uint32_t* device_flags, kvc_stream_t stream);
 
 /* Per-format page pools of one attention layer.  K and V are separate pools
  * that share the block table: logical page j of sequence b lives in slot
@@ -287,15 +295,20 @@ KVC_API kvc_status kvc_exans_workspace_size(int n, int page_size, int n_kv_heads
  *              size plus the header), 16-byte aligned
  *   offsets    device int64 [n + 1], out: blob i is dst[offsets[i],
  *              offsets[i+1]); offsets[n] = the coded size
+ *   n_src_pages  pages in src (>= 1; >= n when page_ids is NULL)
+ *   device_flags device uint32 or NULL: an id outside [0, n_src_pages) is
+ *              checked on the device; its blob codes src page 0 instead (the
+ *              blobs stay back to back) and bit 1 is set
  * Errors: INVALID_ARG (null or misaligned pointers, n outside 0..2^24,
- * dst_bytes too small), WORKSPACE, UNSUPPORTED (page_size != 16, head_dim
- * not 64/128/256, N > 2^22).  Asynchronous on `stream` (three launches:
+ * dst_bytes too small, n_src_pages out of range), WORKSPACE, UNSUPPORTED
+ * (page_size != 16, head_dim not 64/128/256, N > 2^22).  Asynchronous on `stream` (three launches:
  * code into per-page workspace slots, prefix sum of the sizes, compaction);
  * allocates nothing.
  */
 KVC_API kvc_status kvc_exans_encode(const void* src_bf16, const int32_t* page_ids, int n, int page_size,
                                     int n_kv_heads, int head_dim, void* workspace, size_t workspace_bytes,
-                                    void* dst, size_t dst_bytes, int64_t* offsets, kvc_stream_t stream);
+                                    void* dst, size_t dst_bytes, int64_t* offsets, int64_t n_src_pages,
+                                    uint32_t* device_flags, kvc_stream_t stream);
 
 /*
  * kvc_exans_decode - decode blobs back to bf16 pages (bit-exact inverse).
@@ -386,10 +399,12 @@ KVC_API kvc_status kvc_decode_workspace_size(int batch, int n_q_heads, int n_kv_
  *   softmax_scale <= 0 selects 1/sqrt(head_dim)
  *   out           device float32 [batch][Hq][D]
  *   workspace     device, >= kvc_decode_workspace_size() bytes, 256-byte
- *                 aligned; its merge tickets must be zero before the first
- *                 call (zero the whole buffer once); every call leaves them
- *                 zero again, so one workspace serves repeated calls and
- *                 CUDA-graph replay, but not two calls in flight at once.
+ *                 aligned, any contents: each call clears its error word and
+ *                 merge tickets first (one cudaMemsetAsync on `stream`,
+ *                 captured with the kernel in a CUDA graph) and rewrites the
+ *                 partial states, so one workspace serves repeated calls and
+ *                 graph replay, but not two calls in flight at once.  The
+ *                 flags of a call are therefore read before the next call.
  * Device-side checks (block-table entry outside its pool, unknown page
  * format, context length out of range) skip the offending page or
  * sequence and set a flag that kvc_decode_read_error() returns.
@@ -417,6 +432,8 @@ KVC_API kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_page
  *   block_table, older_fmt, context_lens   as for one layer, [batch][...]
  *   out           device float32 [n_layers][batch][Hq][D]
  *   workspace     >= kvc_decode_workspace_size(n_layers * batch, ...) bytes
+ * n_layers * n_pages[f] * n_kv_heads must stay below 2^31 for every format
+ * (KVC_ERR_UNSUPPORTED otherwise).
  * Everything else as kvc_decode_attention_paged, which is this call with
  * n_layers = 1.  INVALID_ARG also for n_layers < 1 or n_layers * batch
  * above 2^30.
@@ -459,7 +476,10 @@ KVC_API kvc_status kvc_decode_read_error(void* workspace, int batch, int n_q_hea
  * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *   - The first call on a device looks up the array's device address on
  *     that device (cudaGetSymbolAddress, with the device current) and caches
- *     it; make that first call before any stream capture.
+ *     it; make that first call before any stream capture.  The cached
+ *     address belongs to that device's primary context: after
+ *     cudaDeviceReset the library must be reloaded (a new process) before
+ *     this entry point is used again on that device.
  *   - Each call clears the error word and the merge tickets with
  *     cudaMemsetAsync on `stream` before the kernel; the partial states are
  *     fully rewritten.

@@ -42,9 +42,9 @@ def test_status_strings():
     assert K.kvc_status_string(99) == "unknown status"
 
 
-def _expect(status, fn, *args):
+def _expect(status, fn, *args, **kw):
     with pytest.raises(K.KvcError) as e:
-        fn(*args)
+        fn(*args, **kw)
     assert e.value.status == status
 
 
@@ -60,6 +60,9 @@ def test_codec_argument_errors_without_gpu():
     _expect(K.KVC_ERR_INVALID_ARG, q, fake, None, 4, 16, 0, 128, K.KVC_FMT_FP8_E4M3, fake, fake)
     _expect(K.KVC_ERR_INVALID_ARG, q, fake, None, 4, 16, 2, 128, 7, fake, fake)
     K.kvc_quantize_pack_pages(None, None, 0, 16, 2, 128, K.KVC_FMT_TERNARY2, None, None)  # n = 0: no-op
+    # the source pool must hold the pages named (ids 0..n-1 when page_ids is NULL)
+    _expect(K.KVC_ERR_INVALID_ARG, q, fake, None, 4, 16, 2, 128, K.KVC_FMT_TERNARY2, fake, fake, n_src_pages=3)
+    _expect(K.KVC_ERR_INVALID_ARG, q, fake, fake, 4, 16, 2, 128, K.KVC_FMT_TERNARY2, fake, fake, n_src_pages=0)
     d = K.kvc_dequantize_pages
     _expect(K.KVC_ERR_UNSUPPORTED, d, fake, fake, None, 4, 16, 2, 32, K.KVC_FMT_TERNARY2, fake)
     _expect(K.KVC_ERR_INVALID_ARG, d, fake, None, None, 4, 16, 2, 64, K.KVC_FMT_FP8_E4M3, fake)
@@ -195,15 +198,17 @@ def test_exans_argument_errors():
     N = 8 * 16 * 128
     ws = 4 * N + 192
 
-    def enc(n=2, ptr=p, ws_bytes=2 * ws, dst_bytes=2 * (64 + 2 * N), d=128):
+    def enc(n=2, ptr=p, ws_bytes=2 * ws, dst_bytes=2 * (64 + 2 * N), d=128, n_src=2):
         return lib.kvc_exans_encode(ptr, None, n, 16, 8, d, ptr, ctypes.c_size_t(ws_bytes), ptr,
-                                    ctypes.c_size_t(dst_bytes), ptr, None)
+                                    ctypes.c_size_t(dst_bytes), ptr, ctypes.c_int64(n_src), None, None)
     assert enc(n=-1) == K.KVC_ERR_INVALID_ARG
     assert enc(d=80) == K.KVC_ERR_UNSUPPORTED
     assert enc(ptr=None) == K.KVC_ERR_INVALID_ARG
     assert enc(ptr=vp((1 << 20) + 8)) == K.KVC_ERR_INVALID_ARG   # misaligned
     assert enc(ws_bytes=2 * ws - 1) == K.KVC_ERR_WORKSPACE
     assert enc(dst_bytes=2 * (64 + 2 * N) - 16) == K.KVC_ERR_INVALID_ARG
+    assert enc(n_src=0) == K.KVC_ERR_INVALID_ARG                  # no source pages
+    assert enc(n_src=1) == K.KVC_ERR_INVALID_ARG                  # ids 0..n-1 need n source pages
     def dec(n=2, ptr=p, d=128):
         return lib.kvc_exans_decode(ptr, ctypes.c_size_t(1 << 20), ptr, 2, None, n, 16, 8, d, ptr, None, None)
     assert dec(n=0) == K.KVC_OK
@@ -216,3 +221,12 @@ def test_layout_version_matches_the_header():
     src = open(os.path.join(ROOT, "include", "kvc.h")).read()
     v = int(re.search(r"#define KVC_LAYOUT_VERSION (\d+)", src).group(1))
     assert K.kvc_layout_version() == v == K.LAYOUT_VERSION
+
+
+def test_noalloc_scratch_size_matches_header():
+    # the binding's copy of KVC_NOALLOC_SCRATCH_BYTES is the header's value
+    import re
+    hdr = open(os.path.join(ROOT, "include", "kvc.h")).read()
+    m = re.search(r"#define\s+KVC_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", hdr)
+    assert m, "KVC_NOALLOC_SCRATCH_BYTES not found in kvc.h"
+    assert int(m.group(1)) << int(m.group(2)) == K.NOALLOC_SCRATCH_BYTES

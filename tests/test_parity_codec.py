@@ -166,3 +166,56 @@ def test_bulk_workload_full_size_sampled(cuda_device):
     q, s = _quant(pages, K.KVC_FMT_FP8_E4M3)
     q_o, s_o = O.quantize_fp8_pages(bits(pages[idx]))
     assert np.array_equal(q[idx].cpu().numpy(), q_o) and np.array_equal(s[idx].cpu().numpy(), s_o)
+
+
+@pytest.mark.parametrize("mode", [K.KVC_FMT_TERNARY2, K.KVC_FMT_FP8_E4M3, K.KVC_FMT_BF16])
+@pytest.mark.parametrize("d", [64, 256])
+def test_bad_page_ids_are_skipped_and_flagged(cuda_device, mode, d):
+    # host-built ids with two entries outside the 9 source pages: those
+    # output pages keep their sentinel bytes, the rest match the oracle's
+    # codec on the pages named, and bit 1 of the flag word is set
+    hkv, n_src = 2, 9
+    src = _rand_pages(n_src, hkv, d, seed=77 + d, dev=cuda_device)
+    ids_h = np.array([3, -1, 0, 8, n_src + 4, 5], dtype=np.int32)
+    ids = torch.from_numpy(ids_h).to(cuda_device)
+    n = len(ids_h)
+    flags = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    if mode == K.KVC_FMT_TERNARY2:
+        dst = torch.full((n, hkv, 16, d // 4), 0xAA, dtype=torch.uint8, device=cuda_device)
+        sc = torch.full((n, hkv), -7.0, device=cuda_device)
+    elif mode == K.KVC_FMT_FP8_E4M3:
+        dst = torch.full((n, hkv, 16, d), 0x7F, dtype=torch.uint8, device=cuda_device)
+        sc = torch.full((n,), -7.0, device=cuda_device)
+    else:
+        dst = torch.full((n, hkv, 16, d), 5.0, dtype=torch.bfloat16, device=cuda_device)
+        sc = None
+    K.kvc_quantize_pack_pages(src, ids, n, 16, hkv, d, mode, dst, sc, n_src_pages=n_src, device_flags=flags)
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 1
+    good = np.array([0 <= i < n_src for i in ids_h])
+    out = dst.cpu()
+    src_b = bits(src)
+    if mode == K.KVC_FMT_TERNARY2:
+        assert (out[~good] == 0xAA).all() and (sc.cpu()[~good] == -7.0).all()
+        check_ternary(out[good].numpy(), sc.cpu()[good].numpy(), src_b[ids_h[good]])
+    elif mode == K.KVC_FMT_FP8_E4M3:
+        assert (out[~good] == 0x7F).all() and (sc.cpu()[~good] == -7.0).all()
+        q_o, s_o = O.quantize_fp8_pages(src_b[ids_h[good]])
+        assert np.array_equal(out[good].numpy(), q_o) and np.array_equal(sc.cpu()[good].numpy(), s_o)
+    else:
+        assert (out[~good].float() == 5.0).all()
+        assert np.array_equal(bits(out[good]), src_b[ids_h[good]])
+    # dequantise from the n compressed pages just made, two ids outside them
+    if mode != K.KVC_FMT_BF16:
+        ids2 = torch.tensor([0, 2, n + 3, -5], dtype=torch.int32, device=cuda_device)
+        rt = torch.full((4, hkv, 16, d), 3.0, dtype=torch.bfloat16, device=cuda_device)
+        flags.zero_()
+        K.kvc_dequantize_pages(dst, sc, ids2, 4, 16, hkv, d, mode, rt, n_src_pages=n, device_flags=flags)
+        torch.cuda.synchronize()
+        assert int(flags.item()) == 1
+        assert (rt.cpu()[2:].float() == 3.0).all()
+        if mode == K.KVC_FMT_TERNARY2:
+            ref = O.dequantize_ternary(out[[0, 2]].numpy(), sc.cpu()[[0, 2]].numpy())
+        else:
+            ref = O.dequantize_fp8(out[[0, 2]].numpy(), sc.cpu()[[0, 2]].numpy())
+        assert np.array_equal(bits(rt[:2]), ref)

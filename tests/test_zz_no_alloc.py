@@ -52,6 +52,42 @@ def test_noalloc_matches_regular_entry_point_twice(cuda_device, name, over):
                                f"{name} no-alloc call {call}")
 
 
+def _setup(name, dev, seed, **over):
+    inp = synth.make_decode_inputs(name, seed=seed, **over)
+    cfg = inp["cfg"]
+    hp = HP[cfg["hp"]]
+    cache, bt, fmt, older = oracle_build_from_inputs(inp, hp)
+    pools, struct = upload_oracle_cache(cache, dev)
+    args = dict(q=inp["q"].to(dev), struct=struct, bt=torch.from_numpy(bt).to(dev),
+                older=lib_older_fmt(older, dev), lens=inp["context_lens"].to(dev), hkv=cfg["n_kv_heads"],
+                max_pages=bt.shape[1], sink=cfg["sink"], window=cfg["window"], hp=hp)
+    return args, pools
+
+
+def _noalloc(a):
+    B, hq, d = a["q"].shape
+    out = torch.full((B, hq, d), float("nan"), dtype=torch.float32, device=a["q"].device)
+    K.kvc_decode_attention_paged_noalloc(a["q"], a["struct"], a["bt"], a["older"], a["lens"], B, hq, a["hkv"], d,
+                                         K.PAGE_SIZE, a["max_pages"], a["sink"], a["window"], a["hp"], 0.0, out)
+    return out
+
+
+def test_noalloc_small_then_large_call(cuda_device):
+    # the first call (4 (sequence, KV head) pairs) leaves partial states at
+    # the start of the array that the second call (96 pairs) uses for its
+    # merge tickets: the second call must clear them before it runs
+    small, ps = _setup("tiny", cuda_device, seed=3)
+    large, pl = _setup("qwen3b", cuda_device, seed=4, batch=48, context=16 * 12 + 5)
+    assert small["q"].shape[0] * small["hkv"] <= 8 and large["q"].shape[0] * large["hkv"] > 64
+    for a in (small, large, small, large):
+        out = _noalloc(a)
+        torch.cuda.synchronize()
+        ref, _ = run_decode(a["q"], a["struct"], a["bt"], a["older"], a["lens"], a["hkv"], a["max_pages"],
+                            a["sink"], a["window"], a["hp"])
+        torch.cuda.synchronize()
+        assert_attention_close(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "no-alloc sequence")
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_device):
     # a workspace larger than the fixed array is refused before any work
     B, hq, hkv, d, max_pages = 4096, 64, 8, 256, 1 << 15
