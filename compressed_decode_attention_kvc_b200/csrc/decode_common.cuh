@@ -308,10 +308,10 @@ __device__ __forceinline__ void meta_phase_a(const DecodeParams& p, const Prolog
   }
   const int g = q * hpc + wi;                      // this warp's KV head
   const int bq = b * (p.Hkv / hpc) + q;            // (sequence, head group) pair
-  int rb = b;                                      // row of the shared block table
-  if (p.Bseq != p.B) {                             // stacked layers (uniform branch)
-    a.layer = b / p.Bseq;
-    rb = b - a.layer * p.Bseq;
+  int rb = p.b_base + b;                           // virtual sequence -> row of the shared block table
+  if (rb >= p.Bseq) {                              // stacked layers
+    a.layer = rb / p.Bseq;
+    rb -= a.layer * p.Bseq;
   }
   const long long row = (long long)rb * p.max_pages + j;
   const int last_valid = min((j + 1) * kPage, L) - 1;

@@ -44,6 +44,7 @@
 
 #include <math.h>
 
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -877,7 +878,8 @@ __global__ void __launch_bounds__(HPC * 32) decode_tc_kernel(DecodeParams p) {
       const int b = base + lane;
       int u = 0, c = 0;
       if (b < p.B) {
-        int L = p.ctx[p.Bseq == p.B ? b : b % p.Bseq];
+        const int gb = p.b_base + b;               // virtual sequence of the whole batch
+        int L = p.ctx[gb < p.Bseq ? gb : gb % p.Bseq];
         if (L < 0 || L > p.max_pages * kPage) {
           if (blockIdx.x == 0) atomicOr(p.err, kErrContext);
           L = 0;
@@ -992,12 +994,14 @@ void launch_tc(const DecodeParams& p, int hpc, int grid, cudaStream_t s) {
 
 }  // namespace
 
-// Largest batch the tensor-core kernel handles (its per-CTA sequence table
-// lives in shared memory); larger batches use the CUDA-core kernel.
-constexpr int kTcMaxBatch = kTcMaxBatchTpl;
-
-bool tc_supported(int batch, int hkv, int max_pages) {
-  return batch <= kTcMaxBatch && (long long)batch * hkv * max_pages * kCostMax < (1ll << 31);
+// Virtual sequences per launch: each CTA keeps the launch's sequence tables
+// in shared memory, so a launch takes at most kTcMaxBatchTpl of them (and
+// few enough that the launch's total page weight fits 31 bits); a larger
+// batch is decoded in consecutive launches of that many.
+int tc_chunk(int hkv, int max_pages) {
+  const long long per = (long long)hkv * std::max(1, max_pages) * kCostMax;
+  const long long fit = ((1ll << 31) - 1) / per;
+  return (int)std::min<long long>(kTcMaxBatchTpl, fit);
 }
 
 // KV heads per CTA: the largest of 4, 2, 1 that divides Hkv.
@@ -1024,16 +1028,30 @@ cudaError_t tc_grid(int batch, int d, int hq, int hkv, int* grid) {
 
 int tc_warps_per_cta(int hkv) { return tc_heads_per_cta(hkv); }
 
-cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s) {
+cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, int chunk, cudaStream_t s) {
   const int hpc = tc_heads_per_cta(p.Hkv);
   const bool narrow = p.G <= 4;
-  switch (head_dim) {
-    case 64: narrow ? launch_tc<64, true>(p, hpc, grid, s) : launch_tc<64, false>(p, hpc, grid, s); break;
-    case 128: narrow ? launch_tc<128, true>(p, hpc, grid, s) : launch_tc<128, false>(p, hpc, grid, s); break;
-    case 256: narrow ? launch_tc<256, true>(p, hpc, grid, s) : launch_tc<256, false>(p, hpc, grid, s); break;
-    default: return cudaErrorInvalidValue;
+  if (chunk < 1) return cudaErrorInvalidValue;
+  // consecutive launches of `chunk` virtual sequences; each launch owns its
+  // rows of Q, the output and the tickets, and reuses the partial records
+  // (the launches run one after another on the stream)
+  for (int b0 = 0; b0 < p.B; b0 += chunk) {
+    DecodeParams c = p;
+    c.b_base = p.b_base + b0;
+    c.B = std::min(chunk, p.B - b0);
+    c.q = p.q + (long long)b0 * p.Hq * head_dim;
+    c.out = p.out + (long long)b0 * p.Hq * head_dim;
+    c.tickets = p.tickets + (long long)b0 * p.Hkv;
+    switch (head_dim) {
+      case 64: narrow ? launch_tc<64, true>(c, hpc, grid, s) : launch_tc<64, false>(c, hpc, grid, s); break;
+      case 128: narrow ? launch_tc<128, true>(c, hpc, grid, s) : launch_tc<128, false>(c, hpc, grid, s); break;
+      case 256: narrow ? launch_tc<256, true>(c, hpc, grid, s) : launch_tc<256, false>(c, hpc, grid, s); break;
+      default: return cudaErrorInvalidValue;
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 }  // namespace kvc

@@ -1267,7 +1267,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) decode_umma_kernel(DecodePara
       const int b = base + lane;
       int u = 0, c = 0;
       if (b < p.B) {
-        int Lb = p.ctx[p.Bseq == p.B ? b : b % p.Bseq];
+        const int gb = p.b_base + b;
+        int Lb = p.ctx[gb < p.Bseq ? gb : gb % p.Bseq];
         if (Lb < 0 || Lb > p.max_pages * kPage) {
           if (blockIdx.x == 0) atomicOr(p.err, kErrContext);
           Lb = 0;

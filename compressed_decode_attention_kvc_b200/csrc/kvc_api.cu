@@ -53,6 +53,7 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
   const long long bg = (long long)batch * hkv;
   const int G = hq / hkv;
   const size_t record = (size_t)G * (d + 2) * sizeof(float);
+  plan->chunk = 0;
   plan->ticket_offset = 256;
   plan->partial_offset = round_up(256 + (size_t)bg * 4, 256);
   if (umma_selected() && umma_supported(batch, d, hkv, max_pages)) {
@@ -68,17 +69,22 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
     plan->bytes = plan->partial_offset + 2 * ((size_t)plan->n_splits + (size_t)bg) * record;
     return cudaSuccess;
   }
-  if (tc_supported(batch, hkv, max_pages)) {
+  const int chunk = tc_chunk(hkv, max_pages);
+  if (chunk >= 1) {
     // persistent grid, every warp a stream-K worker; one partial state per
-    // (warp, pair) boundary: at most warps + pairs records
+    // (warp, pair) boundary: at most warps + pairs records per launch.  A
+    // batch larger than `chunk` runs as consecutive launches that reuse the
+    // records (each has its own tickets).
+    const int per_launch = std::min(batch, chunk);
     int grid = 0;
-    cudaError_t e = tc_grid(batch, d, hq, hkv, &grid);
+    cudaError_t e = tc_grid(per_launch, d, hq, hkv, &grid);
     if (e != cudaSuccess) return e;
     plan->kernel = kDecodeTc;
     plan->grid = grid;
+    plan->chunk = chunk;
     plan->n_splits = grid * tc_warps_per_cta(hkv);
     plan->pages_per_split = 0;
-    plan->bytes = plan->partial_offset + ((size_t)plan->n_splits + (size_t)bg) * record;
+    plan->bytes = plan->partial_offset + ((size_t)plan->n_splits + (size_t)per_launch * hkv) * record;
     return cudaSuccess;
   }
   int dev = 0, sms = 0;
@@ -103,7 +109,7 @@ cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, Decode
 
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const DecodePlan& plan, cudaStream_t s) {
   if (plan.kernel == kDecodeUmma) return launch_decode_umma(p, head_dim, plan.grid, s);
-  if (plan.kernel == kDecodeTc) return launch_decode_tc(p, head_dim, plan.grid, s);
+  if (plan.kernel == kDecodeTc) return launch_decode_tc(p, head_dim, plan.grid, plan.chunk, s);
   return launch_decode_simple(p, head_dim, s);
 }
 
@@ -347,6 +353,23 @@ kvc_status kvc_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads, i
   return KVC_OK;
 }
 
+kvc_status kvc_decode_plan_info(int batch, int n_q_heads, int n_kv_heads, int head_dim, int max_pages,
+                                int32_t* kernel, int32_t* launches) {
+  if (!kernel || !launches || batch < 0 || max_pages < 0 || n_kv_heads < 1 || n_q_heads < 1)
+    return KVC_ERR_INVALID_ARG;
+  if (n_q_heads % n_kv_heads) return KVC_ERR_INVALID_ARG;
+  if (!head_dim_ok(head_dim) || n_q_heads / n_kv_heads > 8) return KVC_ERR_UNSUPPORTED;
+  kvc::DecodePlan plan;
+  if (kvc::decode_plan(batch, n_q_heads, n_kv_heads, head_dim, max_pages, &plan) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  *kernel = plan.kernel == kvc::kDecodeUmma ? KVC_DECODE_KERNEL_TCGEN05
+            : plan.kernel == kvc::kDecodeTc ? KVC_DECODE_KERNEL_MMA : KVC_DECODE_KERNEL_CUDA_CORE;
+  if (batch == 0) *launches = 0;
+  else if (plan.kernel == kvc::kDecodeTc) *launches = (batch + plan.chunk - 1) / plan.chunk;
+  else *launches = 1;
+  return KVC_OK;
+}
+
 kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache* cache,
                                       const int32_t* block_table, const uint8_t* older_fmt,
                                       const int32_t* context_lens, int batch, int n_q_heads,
@@ -414,6 +437,7 @@ kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged
   p.ctx = context_lens;
   p.B = batch;
   p.Bseq = seqs;
+  p.b_base = 0;
   p.Hq = n_q_heads;
   p.Hkv = n_kv_heads;
   p.G = n_q_heads / n_kv_heads;

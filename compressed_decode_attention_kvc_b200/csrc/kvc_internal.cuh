@@ -75,6 +75,9 @@ struct DecodeParams {
   int Bseq;                  // sequences per layer; B = layers * Bseq virtual sequences
                              // (virtual sequence b: layer b / Bseq, sequence b % Bseq;
                              // layer l's pool slots start at l * n_pages[format])
+  int b_base;                // virtual sequence of this launch's entry 0, when a batch
+                             // is decoded in several launches (q, out and tickets
+                             // then point at that entry's rows)
   int sink, window, hp;
   float scale_log2;          // softmax_scale * log2(e)
   int n_splits, pages_per_split;
@@ -89,6 +92,7 @@ struct DecodePlan {
   int n_splits;              // simple: splits per (sequence, KV head); tc: warps in the grid
   int pages_per_split;       // simple only
   int grid;                  // tc only: persistent CTAs
+  int chunk;                 // tc only: virtual sequences per launch
   size_t ticket_offset, partial_offset, bytes;
 };
 
@@ -102,10 +106,12 @@ cudaError_t launch_decode(const DecodeParams& p, int head_dim, const DecodePlan&
 cudaError_t launch_decode_simple(const DecodeParams& p, int head_dim, cudaStream_t s);
 
 // tensor-core kernel (decode_tc.cu)
-bool tc_supported(int batch, int hkv, int max_pages);
+// virtual sequences one launch of the tensor-core kernel takes (a larger
+// batch is decoded in consecutive launches); 0 when these shapes do not fit
+int tc_chunk(int hkv, int max_pages);
 cudaError_t tc_grid(int batch, int d, int hq, int hkv, int* grid);
 int tc_warps_per_cta(int hkv);
-cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, cudaStream_t s);
+cudaError_t launch_decode_tc(const DecodeParams& p, int head_dim, int grid, int chunk, cudaStream_t s);
 
 // tensor-memory (tcgen05) kernel (decode_umma.cu): two partial records per
 // (CTA, sequence, KV head)

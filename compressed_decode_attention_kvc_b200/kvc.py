@@ -45,8 +45,13 @@ EXPORTS = (
     "kvc_plan_paged_cache", "kvc_decode_workspace_size", "kvc_decode_attention_paged",
     "kvc_decode_read_error", "kvc_decode_attention_paged_noalloc", "kvc_append_retier",
     "kvc_decode_attention_paged_layers", "kvc_promote_pages", "kvc_exans_workspace_size",
-    "kvc_exans_encode", "kvc_exans_decode", "kvc_layout_version",
+    "kvc_exans_encode", "kvc_exans_decode", "kvc_layout_version", "kvc_decode_plan_info",
 )
+
+# decode kernels (KVC_DECODE_KERNEL_* of include/kvc.h)
+KVC_DECODE_KERNEL_CUDA_CORE = 0
+KVC_DECODE_KERNEL_MMA = 1
+KVC_DECODE_KERNEL_TCGEN05 = 2
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -100,6 +105,9 @@ def _load() -> ctypes.CDLL:
     lib.kvc_plan_paged_cache.argtypes = [vp, i32, i32, i32, i32, i32, st, vp, vp, vp, vp, vp, vp]
     lib.kvc_decode_workspace_size.restype = st
     lib.kvc_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.kvc_decode_plan_info.restype = st
+    lib.kvc_decode_plan_info.argtypes = [i32, i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(ctypes.c_int32)]
     lib.kvc_decode_attention_paged.restype = st
     lib.kvc_decode_attention_paged.argtypes = [
         vp, ctypes.POINTER(kvc_paged_cache), vp, vp, vp, i32, i32, i32, i32, i32, i32,
@@ -250,6 +258,16 @@ def kvc_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, max_pages)
                                           ctypes.byref(out)),
            "kvc_decode_workspace_size")
     return out.value
+
+
+def kvc_decode_plan_info(batch, n_q_heads, n_kv_heads, head_dim, max_pages) -> tuple:
+    """(kernel, launches): the KVC_DECODE_KERNEL_* a decode call of these
+    shapes runs on the current device, and its launches per call."""
+    kern, launches = ctypes.c_int32(-1), ctypes.c_int32(-1)
+    _check(_lib.kvc_decode_plan_info(batch, n_q_heads, n_kv_heads, head_dim, max_pages,
+                                     ctypes.byref(kern), ctypes.byref(launches)),
+           "kvc_decode_plan_info")
+    return kern.value, launches.value
 
 
 def make_paged_cache(k_bf16=None, v_bf16=None, k_fp8=None, v_fp8=None, k_fp8_scale=None,

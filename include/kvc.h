@@ -376,6 +376,28 @@ KVC_API kvc_status kvc_plan_paged_cache(const int32_t* context_lens, int batch, 
 KVC_API kvc_status kvc_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads, int head_dim,
                                      int max_pages, size_t* bytes);
 
+/* Decode kernels (kvc_decode_plan_info's *kernel). */
+#define KVC_DECODE_KERNEL_CUDA_CORE 0   /* CUDA-core fallback: shapes the others do not take */
+#define KVC_DECODE_KERNEL_MMA 1         /* tensor-core kernel (register-sourced MMAs), the default */
+#define KVC_DECODE_KERNEL_TCGEN05 2     /* tensor-memory kernel, opt-in (KVC_DECODE_KERNEL=tcgen05) */
+
+/*
+ * kvc_decode_plan_info - which kernel kvc_decode_attention_paged runs for
+ * these shapes on the current device, and in how many launches (a batch
+ * above the tensor-core kernel's per-launch limit of 1024 virtual sequences
+ * is decoded in consecutive launches).  Host only; enqueues nothing.
+ *
+ *   batch     virtual sequences of the call (n_layers * batch for
+ *             kvc_decode_attention_paged_layers)
+ *   kernel    host int32 out: a KVC_DECODE_KERNEL_* value
+ *   launches  host int32 out: kernel launches per call (0 for batch 0)
+ *
+ * Errors: as kvc_decode_workspace_size; KVC_ERR_INVALID_ARG for a NULL
+ * output pointer.
+ */
+KVC_API kvc_status kvc_decode_plan_info(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                        int max_pages, int32_t* kernel, int32_t* launches);
+
 /*
  * kvc_decode_attention_paged - one query token per sequence attends to its
  * whole mixed-format paged cache (Minima, "How mixed-format attention

@@ -230,3 +230,21 @@ def test_noalloc_scratch_size_matches_header():
     m = re.search(r"#define\s+KVC_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", hdr)
     assert m, "KVC_NOALLOC_SCRATCH_BYTES not found in kvc.h"
     assert int(m.group(1)) << int(m.group(2)) == K.NOALLOC_SCRATCH_BYTES
+
+
+def test_decode_plan_info_argument_errors_and_constants():
+    lib = K.kvc._lib
+    import ctypes
+    one = ctypes.c_int32(0)
+    assert lib.kvc_decode_plan_info(2, 8, 2, 128, 10, None, ctypes.byref(one)) == K.KVC_ERR_INVALID_ARG
+    assert lib.kvc_decode_plan_info(2, 8, 2, 128, 10, ctypes.byref(one), None) == K.KVC_ERR_INVALID_ARG
+    _expect(K.KVC_ERR_INVALID_ARG, K.kvc_decode_plan_info, 2, 8, 3, 128, 10)
+    _expect(K.KVC_ERR_INVALID_ARG, K.kvc_decode_plan_info, -1, 8, 2, 128, 10)
+    _expect(K.KVC_ERR_UNSUPPORTED, K.kvc_decode_plan_info, 2, 18, 2, 128, 10)
+    _expect(K.KVC_ERR_UNSUPPORTED, K.kvc_decode_plan_info, 2, 8, 2, 96, 10)
+    # the binding's kernel ids are the header's
+    hdr = open(os.path.join(ROOT, "include", "kvc.h")).read()
+    ids = dict((m.group(1), int(m.group(2)))
+               for m in re.finditer(r"#define\s+(KVC_DECODE_KERNEL_\w+)\s+(\d+)", hdr))
+    assert ids == {n: getattr(K, n) for n in ("KVC_DECODE_KERNEL_CUDA_CORE", "KVC_DECODE_KERNEL_MMA",
+                                                "KVC_DECODE_KERNEL_TCGEN05")}

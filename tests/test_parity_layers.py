@@ -5,8 +5,8 @@ is built by the oracle from its own data with the shared page placement
 stacked layer after layer, and every layer's output must match the oracle's
 attention over that layer's pages (max-abs 2e-3, relative-L2 1e-3).  The
 tensor-core kernel is compared in the GQA <= 4 and wider layouts and with
-FP8 / BF16 windows and anchors; a large virtual batch covers the CUDA-core
-kernel."""
+FP8 / BF16 windows and anchors; virtual batches above one launch's 1024
+sequences cover the consecutive launches."""
 
 import numpy as np
 import pytest
@@ -76,9 +76,17 @@ def test_layers_match_oracle_per_layer(cuda_device, name, over, n_layers):
     _run(name, over, n_layers, cuda_device)
 
 
-def test_layers_large_virtual_batch_cuda_core_kernel(cuda_device):
-    # layers * batch above the tensor-core kernel's batch limit (1024)
-    _run("tiny", dict(batch=260, context=64, window=16), 4, cuda_device)
+@pytest.mark.parametrize("batch,n_layers,launches", [
+    (260, 4, 2),      # 1040 entries: the second launch starts inside layer 3 (row 244)
+    (512, 4, 2),      # 2048 entries
+    (700, 3, 3),      # 2100 entries: launches start inside layers 1 and 2
+])
+def test_layers_large_virtual_batch_tensor_core_kernel(cuda_device, batch, n_layers, launches):
+    # layers * batch above one launch's 1024 virtual sequences: the
+    # tensor-core kernel runs in consecutive launches
+    kern, n = K.kvc_decode_plan_info(n_layers * batch, 8, 4, 64, 4)
+    assert (kern, n) == (K.KVC_DECODE_KERNEL_MMA, launches)
+    _run("tiny", dict(batch=batch, context=64, window=16), n_layers, cuda_device)
 
 
 def test_qwen3b_36_layers_full_size_sampled(cuda_device):
