@@ -196,6 +196,9 @@ struct Worker {
       d.ks[k] = cur.ks;
       d.vs[k] = cur.vs;
     }
+    // largest V scale of the entry (scales are >= 0: their bits order as unsigned)
+    const uint32_t vmax = __reduce_max_sync(kFull, mine ? __float_as_uint(cur.vs) : 0u);
+    if (lane == li) d.gvmax = __uint_as_float(vmax);
     __syncwarp();
     if (copy) {
       // the HPC heads' groups of a page are contiguous: one copy per page
@@ -494,16 +497,23 @@ struct Worker {
     m23 = (t0 + 8 < nt ? 0x0000FFFFu : 0u) | (t0 + 9 < nt ? 0xFFFF0000u : 0u);
   }
 
+  // Threads with tig >= 2 read their token pairs in the order (2tig + 1, 2tig)
+  // so that no two lanes of a load share a bank, and swap the two halves of
+  // their P^T fragments to match.
   __device__ __forceinline__ void pv_ternary(const unsigned char* vg, uint32_t b0, uint32_t b1, int nt) {
-    const int t0 = 2 * tig;
+    const int sw = tig >> 1;
+    const int ta = 2 * tig + sw, tb = 2 * tig + 1 - sw;   // tokens of the low and high f16 halves
+    const uint32_t hsel = sw ? 0x1032u : 0x3210u;
+    b0 = prmt(b0, b0, hsel);
+    b1 = prmt(b1, b1, hsel);
     const int vw0 = (gid * S::kUPT) >> 1;
     uint32_t w0[S::kVW], w1[S::kVW], w2[S::kVW], w3[S::kVW];
 #pragma unroll
     for (int i = 0; i < S::kVW; ++i) {
-      w0[i] = lds<uint32_t>(vg + t0 * (D / 4) + 4 * (vw0 + i));
-      w1[i] = lds<uint32_t>(vg + (t0 + 1) * (D / 4) + 4 * (vw0 + i));
-      w2[i] = lds<uint32_t>(vg + (t0 + 8) * (D / 4) + 4 * (vw0 + i));
-      w3[i] = lds<uint32_t>(vg + (t0 + 9) * (D / 4) + 4 * (vw0 + i));
+      w0[i] = lds<uint32_t>(vg + ta * (D / 4) + 4 * (vw0 + i));
+      w1[i] = lds<uint32_t>(vg + tb * (D / 4) + 4 * (vw0 + i));
+      w2[i] = lds<uint32_t>(vg + (ta + 8) * (D / 4) + 4 * (vw0 + i));
+      w3[i] = lds<uint32_t>(vg + (tb + 8) * (D / 4) + 4 * (vw0 + i));
     }
     uint32_t r01[S::kUPT], r23[S::kUPT];
 #pragma unroll
@@ -515,8 +525,8 @@ struct Worker {
       r23[ul] = prmt(w2[wi], w3[wi], sel);
     }
     if (nt < kPage) {
-      uint32_t m01, m23;
-      pv_masks(nt, m01, m23);
+      const uint32_t m01 = (ta < nt ? 0x0000FFFFu : 0u) | (tb < nt ? 0xFFFF0000u : 0u);
+      const uint32_t m23 = (ta + 8 < nt ? 0x0000FFFFu : 0u) | (tb + 8 < nt ? 0xFFFF0000u : 0u);
 #pragma unroll
       for (int ul = 0; ul < S::kUPT; ++ul) { r01[ul] &= m01; r23[ul] &= m23; }
     }
@@ -583,6 +593,162 @@ struct Worker {
       }
       mma16816_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
       if constexpr (!NARROW) mma16816_bf16(acc[mt], a0, a1, a2, a3, lo0, lo1);
+    }
+  }
+
+  // ---------------------------------- ternary pages, P.V on int8 (NARROW)
+  // With at most 4 query heads a page pair (32 tokens) is one int8 MMA of
+  // k = 32: V^T codes as A (tern8: 64 * code), P as B in two exact unsigned
+  // digits, P ~= (256 * hi + lo) / 2^15 with P = p * gamma_v / gmax <= 1, hi in
+  // column 2h and lo in column 2h + 1.  The int32 sums are exact; they are
+  // folded into the float accumulators once per entry.  Token order along k
+  // (both pages): (2t, 2t + 8, 2t + 1, 2t + 9) for t = tig, the order one
+  // movmatrix of the (token gid, token gid + 8) digit pairs produces.
+  static constexpr int kBB = 2 * S::kUPT;          // bytes of a V row this thread reads
+
+  // The thread's byte block of V rows 2tig, 2tig + 8, 2tig + 1, 2tig + 9 of a
+  // page, transposed: T[b] holds byte b of the four rows in that order.
+  // Threads with tig >= 2 read (and order) 2tig + 1, 2tig + 9, 2tig, 2tig + 8
+  // instead, so that no two lanes of a load share a bank; their P digits are
+  // swapped to match (pv_digits).
+  __device__ __forceinline__ void v_rows_t(const unsigned char* vg, uint32_t (&T)[kBB < 4 ? 4 : kBB]) {
+    constexpr int NW = kBB < 4 ? 1 : kBB / 4;
+    uint32_t r[4][NW];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int tok = 2 * tig + ((q & 1) ? 8 : 0) + ((q >> 1) ^ (tig >> 1));
+      const unsigned char* src = vg + tok * (D / 4) + kBB * gid;
+      if constexpr (kBB == 2) {
+        r[q][0] = lds<uint16_t>(src);
+      } else if constexpr (kBB == 4) {
+        r[q][0] = lds<uint32_t>(src);
+      } else {
+        const uint2 v = lds<uint2>(src);
+        r[q][0] = v.x;
+        r[q][1] = v.y;
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t x01 = prmt(r[0][w], r[1][w], 0x5140u), x23 = prmt(r[0][w], r[1][w], 0x7362u);
+      const uint32_t y01 = prmt(r[2][w], r[3][w], 0x5140u), y23 = prmt(r[2][w], r[3][w], 0x7362u);
+      T[4 * w + 0] = prmt(x01, y01, 0x5410u);
+      T[4 * w + 1] = prmt(x01, y01, 0x7632u);
+      T[4 * w + 2] = prmt(x23, y23, 0x5410u);
+      T[4 * w + 3] = prmt(x23, y23, 0x7632u);
+    }
+  }
+
+  // Rescale of the digit sums by 2^-k (k >= 1): v = 256 hi + lo, floor(v / 2^k).
+  // Within one entry (at most 8 pages) |hi| < 2^20 and |lo| < 2^21, so v
+  // fits 31 bits.
+  __device__ __forceinline__ static void shift_digits(int& hi, int& lo, int k) {
+    const int w = (hi * 256 + lo) >> (k < 31 ? k : 31);
+    hi = w >> 8;
+    lo = w & 255;
+  }
+
+  __device__ __forceinline__ void process_ternary_int(const unsigned char* e, const Desc& d) {
+    constexpr int GB = HPC * group_bytes(KVC_FMT_TERNARY2, D);   // page stride
+    constexpr int NT = kBB < 4 ? 4 : kBB;
+    e += wi * group_bytes(KVC_FMT_TERNARY2, D);
+    const int np = d.np;
+    const float gmax = d.gvmax;
+    if (uref == 0.f && gmax > 0.f) {
+      uref = gmax;
+      inv_uref = 1.f / gmax;
+    }
+    const float r15 = gmax > 0.f ? 32768.f / gmax : 0.f;
+    constexpr float kMagic = 12582912.f;     // 1.5 * 2^23: the low bits of x + kMagic hold round(x)
+    int ai[S::kSteps][4];
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ai[mt][c] = 0;
+    float sA[4], sB[4] = {0.f, 0.f, 0.f, 0.f};
+    qk_ternary(e, sA);
+    if (np > 1) qk_ternary(e + GB, sB);
+    for (int i = 0; i < np; i += 2) {
+      const bool hasB = i + 1 < np;
+      // the next pair's scores, independent of this pair's softmax and P.V
+      float nA[4] = {0.f, 0.f, 0.f, 0.f}, nB[4] = {0.f, 0.f, 0.f, 0.f};
+      if (i + 2 < np) {
+        qk_ternary(e + (i + 2) * GB, nA);
+        if (i + 3 < np) qk_ternary(e + (i + 3) * GB, nB);
+      }
+      uint32_t TA[NT], TB[NT];
+      v_rows_t(e + S::kHalf + i * GB, TA);
+      if (hasB) {
+        v_rows_t(e + S::kHalf + (i + 1) * GB, TB);
+      } else {
+#pragma unroll
+        for (int b = 0; b < NT; ++b) TB[b] = TA[b];   // any finite operand: its P digits are 0
+      }
+      const float scA = d.ks[i] * kq0, scB = hasB ? d.ks[i + 1] * kq0 : 0.f;
+      float x0 = sA[0] * scA, x1 = sA[2] * scA, x2 = sB[0] * scB, x3 = sB[2] * scB;
+      if (i + 2 >= np) {                      // the entry's last pair: masks
+        const int ntA = hasB ? kPage : d.nrows, ntB = hasB ? d.nrows : 0;
+        if (gid >= ntA) x0 = -INFINITY;
+        if (gid + 8 >= ntA) x1 = -INFINITY;
+        if (gid >= ntB) x2 = -INFINITY;
+        if (gid + 8 >= ntB) x3 = -INFINITY;
+      }
+      const float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+      // P <= 1 needs every score at or below the running maximum; the
+      // maximum moves by a whole number k of log2 units, so the digit sums
+      // rescale exactly by a shift
+      if (__any_sync(kFull, mx > m0)) {
+        float r = mx;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) r = fmaxf(r, __shfl_xor_sync(kFull, r, o));
+        if (r > m0) {
+          if (m0 == -INFINITY) {
+            m0 = ceilf(r);
+          } else {
+            const int k = (int)ceilf(r - m0);
+            const float a = k < 126 ? __int_as_float((127 - k) << 23) : 0.f;   // 2^-k
+#pragma unroll
+            for (int mt = 0; mt < S::kSteps; ++mt) {
+              shift_digits(ai[mt][0], ai[mt][1], k);
+              shift_digits(ai[mt][2], ai[mt][3], k);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) acc[mt][c] *= a;
+            }
+            l0 *= a;
+            m0 += (float)k;
+          }
+        }
+      }
+      const float mm = m0 == -INFINITY ? 0.f : m0;
+      const float p0 = ex2(x0 - mm), p1 = ex2(x1 - mm), p2 = ex2(x2 - mm), p3 = ex2(x3 - mm);
+      l0 += (p0 + p1) + (p2 + p3);
+      const float rA = d.vs[i] * r15, rB = hasB ? d.vs[i + 1] * r15 : 0.f;
+      const uint32_t f0 = __float_as_uint(fmaf(p0, rA, kMagic)), f1 = __float_as_uint(fmaf(p1, rA, kMagic));
+      const uint32_t f2 = __float_as_uint(fmaf(p2, rB, kMagic)), f3 = __float_as_uint(fmaf(p3, rB, kMagic));
+      // (hi of token gid, hi of token gid + 8 | lo, lo) -> column (head, digit);
+      // threads with tig >= 2 swap their two token pairs (see v_rows_t)
+      const uint32_t sw = tig >= 2 ? 0x1032u : 0x3210u;
+      const uint32_t t0 = movtrans(prmt(f0, f1, 0x4051u)), t1 = movtrans(prmt(f2, f3, 0x4051u));
+      const uint32_t b0 = prmt(t0, t0, sw), b1 = prmt(t1, t1, sw);
+#pragma unroll
+      for (int mt = 0; mt < S::kSteps; ++mt) {
+        const int lb = mt + S::kSteps;
+        const int blo = 2 * (mt >> 3) + ((mt & 7) >> 2), bhi = 2 * (lb >> 3) + ((lb & 7) >> 2);
+        const int f = mt & 3;
+        imma16832_su(ai[mt], tern8(TA[blo], f), tern8(TA[bhi], f), tern8(TB[blo], f), tern8(TB[bhi], f), b0, b1);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        sA[c] = nA[c];
+        sB[c] = nB[c];
+      }
+    }
+    // sum = gmax * 2^-15 * (256 hi + lo) / 64 (tern8 carries 64 * code)
+    const float cf = gmax * (1.f / 2097152.f) * inv_uref;
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt) {
+      acc[mt][0] += (float)(ai[mt][0] * 256 + ai[mt][1]) * cf;
+      acc[mt][2] += (float)(ai[mt][2] * 256 + ai[mt][3]) * cf;
     }
   }
 
@@ -729,7 +895,9 @@ struct Worker {
   __device__ __forceinline__ void process(const unsigned char* e, const Desc& d) {
     const int fmt = d.fmt, np = d.np;
     uint32_t b0, b1, lo0 = 0u, lo1 = 0u;
-    if (fmt == KVC_FMT_TERNARY2) {
+    if (NARROW && fmt == KVC_FMT_TERNARY2 && p.tern_int) {
+      process_ternary_int(e, d);
+    } else if (fmt == KVC_FMT_TERNARY2) {
       constexpr int GB = HPC * group_bytes(KVC_FMT_TERNARY2, D);   // page stride
       e += wi * group_bytes(KVC_FMT_TERNARY2, D);
       rebase_value_scale(d, 0.5f);

@@ -75,7 +75,12 @@ struct EncSmem {
 // One warp per group; the group's blob is built in its workspace slot of
 // 4N + 192 bytes: header, sign+mantissa bytes, escape area (N), and a stream
 // area (2N + 128 bytes, the most 2 bytes per symbol can take) written
-// backwards from its end, then moved down behind the escapes.
+// backwards from its end, then moved down behind the escapes.  Pass 1 also
+// keeps each value's exponent byte at the front of the stream area, so the
+// later passes read N bytes instead of the 2N of the page: after the chunks
+// from c on are coded the stream holds at most 256 bytes per chunk, and its
+// front (at or above offset 2N + 192 + 256c) never reaches the exponents of
+// the chunks before c (which end at 2N + 64 + 128c).
 __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint16_t* __restrict__ src,
                                                                     const int32_t* __restrict__ page_ids,
                                                                     long long n_src, uint32_t* flags,
@@ -99,22 +104,26 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint1
   if (lane < 16) S.cnt[lane] = 0u;
   __syncwarp();
 
-  // pass 1: exponent histogram; sign+mantissa bytes (chunks is a multiple
-  // of 8; four chunks' loads are issued together)
+  // pass 1: exponent histogram; sign+mantissa bytes; exponent bytes kept
+  // for passes 2 and 3 (chunks is a multiple of 8; four chunks' loads are
+  // issued together)
+  uint32_t* xe = reinterpret_cast<uint32_t*>(slot + kExHeader + 2 * N);
   for (int c0 = 0; c0 < chunks; c0 += 4) {
     uint2 vq[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) vq[k] = *reinterpret_cast<const uint2*>(x + (long long)(c0 + k) * 128 + 4 * lane);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      uint32_t smw = 0;
+      uint32_t smw = 0, ew = 0;
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const uint32_t b = quad_elem(vq[k], r);
         atomicAdd(&S.hist[(b >> 7) & 0xFFu], 1u);
         smw |= (((b >> 8) & 0x80u) | (b & 0x7Fu)) << (8 * r);
+        ew |= ((b >> 7) & 0xFFu) << (8 * r);
       }
       *reinterpret_cast<uint32_t*>(slot + kExHeader + (long long)(c0 + k) * 128 + 4 * lane) = smw;
+      xe[(long long)(c0 + k) * 32 + lane] = ew;
     }
   }
   __syncwarp();
@@ -128,17 +137,16 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint1
   unsigned char* esc_out = slot + kExHeader + N;
   long long esc_base = 0;
   for (int c0 = 0; c0 < chunks; c0 += 4) {
-   uint2 vq[4];
+   uint32_t eq[4];
 #pragma unroll
-   for (int k = 0; k < 4; ++k) vq[k] = *reinterpret_cast<const uint2*>(x + (long long)(c0 + k) * 128 + 4 * lane);
+   for (int k = 0; k < 4; ++k) eq[k] = xe[(long long)(c0 + k) * 32 + lane];
 #pragma unroll
    for (int k = 0; k < 4; ++k) {
-    const uint2 v = vq[k];
     uint32_t e[4];
     int s[4], nesc = 0;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      e[r] = (quad_elem(v, r) >> 7) & 0xFFu;
+      e[r] = (eq[k] >> (8 * r)) & 0xFFu;
       s[r] = symbol_of(e[r], centre);
       atomicAdd(&S.cnt[s[r]], 1u);
       nesc += s[r] == kExEscape;
@@ -190,15 +198,14 @@ __global__ void __launch_bounds__(kExWarps * 32) exans_encode_kernel(const uint1
   long long written = 0;                     // warp-uniform
   uint32_t st = kExL;
   for (int c0 = chunks - 4; c0 >= 0; c0 -= 4) {
-   uint2 vq[4];
+   uint32_t eq[4];
 #pragma unroll
-   for (int k = 0; k < 4; ++k) vq[k] = *reinterpret_cast<const uint2*>(x + (long long)(c0 + k) * 128 + 4 * lane);
+   for (int k = 0; k < 4; ++k) eq[k] = xe[(long long)(c0 + k) * 32 + lane];
 #pragma unroll
    for (int k = 3; k >= 0; --k) {
-    const uint2 v = vq[k];
 #pragma unroll
     for (int r = 3; r >= 0; --r) {
-      const int s = symbol_of((quad_elem(v, r) >> 7) & 0xFFu, centre);
+      const int s = symbol_of((eq[k] >> (8 * r)) & 0xFFu, centre);
       const uint32_t fc = S.fc[s];
       const uint32_t f = fc & 0xFFFFu, cum = fc >> 16;
       const uint32_t xmax = f << (23 - kExScaleBits + 8);

@@ -49,6 +49,17 @@ static bool umma_selected() {
   return on;
 }
 
+// Ternary P.V of the tensor-core kernel at GQA <= 4: int8 MMAs with P in two
+// exact digits (default), or f16 MMAs with P as an f16 hi + lo pair when the
+// environment variable KVC_DECODE_TERNARY_PV is "f16" (read once per process).
+static bool ternary_pv_int() {
+  static const bool on = [] {
+    const char* v = getenv("KVC_DECODE_TERNARY_PV");
+    return v == nullptr || strcmp(v, "f16") != 0;
+  }();
+  return on;
+}
+
 cudaError_t decode_plan(int batch, int hq, int hkv, int d, int max_pages, DecodePlan* plan) {
   const long long bg = (long long)batch * hkv;
   const int G = hq / hkv;
@@ -447,6 +458,7 @@ kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged
   p.hp = hp_mode;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.tern_int = kvc::ternary_pv_int() ? 1 : 0;
   p.n_splits = plan.n_splits;
   p.pages_per_split = plan.pages_per_split;
   p.out = out;

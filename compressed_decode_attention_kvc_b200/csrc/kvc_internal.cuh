@@ -80,6 +80,7 @@ struct DecodeParams {
                              // then point at that entry's rows)
   int sink, window, hp;
   float scale_log2;          // softmax_scale * log2(e)
+  int tern_int;              // tensor-core kernel, GQA <= 4: ternary P.V on int8 MMAs
   int n_splits, pages_per_split;
   float* out;
   uint32_t* err;             // device error word
