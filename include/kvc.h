@@ -430,6 +430,12 @@ KVC_API kvc_status kvc_decode_plan_info(int batch, int n_q_heads, int n_kv_heads
  * Device-side checks (block-table entry outside its pool, unknown page
  * format, context length out of range) skip the offending page or
  * sequence and set a flag that kvc_decode_read_error() returns.
+ * Arithmetic: products on tensor cores, sums in fp32 (ternary pages at
+ * GQA <= 4: exact int32 sums of P's two 8-bit digits, P relative to the
+ * running maximum, 2^-15 steps).  Environment, read once per process:
+ * KVC_DECODE_KERNEL=tcgen05 selects the tensor-memory kernel;
+ * KVC_DECODE_TERNARY_PV=f16 runs the ternary pages' P.V at GQA <= 4 on f16
+ * MMAs (P as an f16 hi + lo pair) instead.
  */
 KVC_API kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache* cache,
                                       const int32_t* block_table, const uint8_t* older_fmt,

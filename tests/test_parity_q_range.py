@@ -96,3 +96,31 @@ def test_bf16_page_beyond_f16_range(cuda_device, d):
     assert float(diff.max()) <= 2e-3 * scale, float(diff.max())
     rel = float(np.linalg.norm(diff)) / float(np.linalg.norm(ref))
     assert rel <= 1e-3, rel
+
+
+@pytest.mark.parametrize("ramp", ["rising", "sawtooth"])
+@pytest.mark.parametrize("d,hq,hkv", [(64, 8, 4), (128, 16, 4), (256, 8, 4), (128, 16, 2)])
+def test_moving_maximum_matches_oracle(cuda_device, d, hq, hkv, ramp):
+    # keys built so that the scores keep rising along the sequence (or rise
+    # and fall back every few pages): the running maximum moves on almost
+    # every page, so the kernel rescales its partial sums many times after
+    # they have accumulated (the digit sums of the int8 P.V path by exact
+    # shifts, the fp32 sums by powers of two)
+    inp = synth.make_decode_inputs("tiny", seed=3 + d + hq, batch=2, n_q_heads=hq, n_kv_heads=hkv,
+                                   head_dim=d, context=16 * 40 + 7, window=20, sink=4, hp="bf16")
+    q = inp["q"].float()
+    k = inp["k_pages"].float()
+    B, max_pages, _, P, _ = k.shape
+    g = hq // hkv
+    # the mean query direction of each KV head's group
+    u = q.view(B, hkv, g, d).mean(dim=2)
+    u = u / u.norm(dim=-1, keepdim=True)
+    pos = torch.arange(max_pages * P, dtype=torch.float32).view(max_pages, P) / (max_pages * P)
+    if ramp == "sawtooth":
+        pos = torch.remainder(pos * 7.0, 1.0)
+    amp = 6.0 * d ** 0.5                      # ~+6 score units per unit of pos per |q| along u
+    k += amp * pos.view(1, max_pages, 1, P, 1) * u.view(B, 1, hkv, 1, d)
+    inp["k_pages"] = k.to(torch.bfloat16)
+    out, ref, flags = _run(inp, cuda_device)
+    assert flags == 0
+    assert_attention_close(out, ref, f"{ramp} D={d} G={g}")
