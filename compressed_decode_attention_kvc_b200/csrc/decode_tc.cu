@@ -71,9 +71,13 @@ __host__ __device__ constexpr int cost_hp(int fmt) {
 
 // HPC: KV heads per CTA (1, 2 or 4), one warp each.  The warps of a CTA walk
 // the same pages; a ring slot holds those pages for all HPC heads.
+// A ring entry holds 8 KB per head (4 KB at head_dim 64).  Two-head CTAs at
+// head_dim 128 (CTAs of 64 threads, six per SM by registers) take 7 KB, so
+// that six of them also fit the shared memory with the sequence tables of a
+// few hundred sequences (a BF16 page then fills two half-page entries).
 template <int D, int HPC>
 struct Shape {
-  static constexpr int kEntryBytes = D == 64 ? 4096 : 8192;   // per head
+  static constexpr int kEntryBytes = D == 64 ? 4096 : (D == 128 && HPC == 2 ? 7168 : 8192);   // per head
   static constexpr int kHeadHalf = kEntryBytes / 2;         // K (or V) bytes of one head per slot
   static constexpr int kSlotBytes = HPC * kEntryBytes;      // one ring slot of the CTA
   static constexpr int kHalf = kSlotBytes / 2;              // K region | V region
