@@ -121,6 +121,7 @@ struct Worker {
   bool nxt_b_pending;       // nxt still needs phase B (its phase A loads are in nxa)
   bool nxa_pending;         // nxa still needs phase A (the chunk after nxt)
   int W;
+  uint32_t wait_limit;      // tries of a bounded slot wait
 
   // per (sequence, KV head) state
   int cur_bg;
@@ -756,6 +757,93 @@ struct Worker {
     }
   }
 
+  // A full entry of 8 ternary pages (the ring's capacity at head_dim 64 and
+  // 128): the scores of all 8 pages first, one test of the running maximum
+  // for the whole entry, then the four page pairs' P.V as one straight run
+  // of code, so the loads, transposes and MMAs of one pair overlap the
+  // softmax of the next.  Same arithmetic as process_ternary_int.
+  __device__ __forceinline__ void process_ternary_int8(const unsigned char* e, const Desc& d) {
+    constexpr int GB = HPC * group_bytes(KVC_FMT_TERNARY2, D);   // page stride
+    constexpr int NT = kBB < 4 ? 4 : kBB;
+    e += wi * group_bytes(KVC_FMT_TERNARY2, D);
+    const float gmax = d.gvmax;
+    if (uref == 0.f && gmax > 0.f) {
+      uref = gmax;
+      inv_uref = 1.f / gmax;
+    }
+    const float r15 = gmax > 0.f ? 32768.f / gmax : 0.f;
+    constexpr float kMagic = 12582912.f;
+    float x[8][2];
+#pragma unroll
+    for (int pg = 0; pg < 8; ++pg) {
+      float s[4];
+      qk_ternary(e + pg * GB, s);
+      const float sc = d.ks[pg] * kq0;
+      x[pg][0] = s[0] * sc;
+      x[pg][1] = s[2] * sc;
+    }
+    // only the entry's last page can be partial
+    if (gid >= d.nrows) x[7][0] = -INFINITY;
+    if (gid + 8 >= d.nrows) x[7][1] = -INFINITY;
+    float mx = x[0][0];
+#pragma unroll
+    for (int pg = 0; pg < 8; ++pg) mx = fmaxf(mx, fmaxf(x[pg][0], x[pg][1]));
+    int ai[S::kSteps][4];
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ai[mt][c] = 0;
+    if (__any_sync(kFull, mx > m0)) {
+      float r = mx;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) r = fmaxf(r, __shfl_xor_sync(kFull, r, o));
+      if (r > m0) {
+        if (m0 == -INFINITY) {
+          m0 = ceilf(r);
+        } else {
+          const int k = (int)ceilf(r - m0);
+          const float a = k < 126 ? __int_as_float((127 - k) << 23) : 0.f;   // 2^-k
+#pragma unroll
+          for (int mt = 0; mt < S::kSteps; ++mt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[mt][c] *= a;
+          l0 *= a;
+          m0 += (float)k;
+        }
+      }
+    }
+    const float mm = m0 == -INFINITY ? 0.f : m0;
+    const uint32_t sw = tig >= 2 ? 0x1032u : 0x3210u;
+#pragma unroll
+    for (int pr2 = 0; pr2 < 4; ++pr2) {
+      const int i = 2 * pr2;
+      uint32_t TA[NT], TB[NT];
+      v_rows_t(e + S::kHalf + i * GB, TA);
+      v_rows_t(e + S::kHalf + (i + 1) * GB, TB);
+      const float p0 = ex2(x[i][0] - mm), p1 = ex2(x[i][1] - mm);
+      const float p2 = ex2(x[i + 1][0] - mm), p3 = ex2(x[i + 1][1] - mm);
+      l0 += (p0 + p1) + (p2 + p3);
+      const float rA = d.vs[i] * r15, rB = d.vs[i + 1] * r15;
+      const uint32_t f0 = __float_as_uint(fmaf(p0, rA, kMagic)), f1 = __float_as_uint(fmaf(p1, rA, kMagic));
+      const uint32_t f2 = __float_as_uint(fmaf(p2, rB, kMagic)), f3 = __float_as_uint(fmaf(p3, rB, kMagic));
+      const uint32_t t0 = movtrans(prmt(f0, f1, 0x4051u)), t1 = movtrans(prmt(f2, f3, 0x4051u));
+      const uint32_t b0 = prmt(t0, t0, sw), b1 = prmt(t1, t1, sw);
+#pragma unroll
+      for (int mt = 0; mt < S::kSteps; ++mt) {
+        const int lb = mt + S::kSteps;
+        const int blo = 2 * (mt >> 3) + ((mt & 7) >> 2), bhi = 2 * (lb >> 3) + ((lb & 7) >> 2);
+        const int f = mt & 3;
+        imma16832_su(ai[mt], tern8(TA[blo], f), tern8(TA[bhi], f), tern8(TB[blo], f), tern8(TB[bhi], f), b0, b1);
+      }
+    }
+    const float cf = gmax * (1.f / 2097152.f) * inv_uref;
+#pragma unroll
+    for (int mt = 0; mt < S::kSteps; ++mt) {
+      acc[mt][0] += (float)(ai[mt][0] * 256 + ai[mt][1]) * cf;
+      acc[mt][2] += (float)(ai[mt][2] * 256 + ai[mt][3]) * cf;
+    }
+  }
+
   // --------------------------------------------------- softmax, per page
   // Scales the score tile, applies the row mask, moves the lazy maximum when
   // needed, accumulates the row sums and returns P^T fragments (P scaled by
@@ -900,7 +988,8 @@ struct Worker {
     const int fmt = d.fmt, np = d.np;
     uint32_t b0, b1, lo0 = 0u, lo1 = 0u;
     if (NARROW && fmt == KVC_FMT_TERNARY2 && p.tern_int) {
-      process_ternary_int(e, d);
+      if (S::kTernCap == 8 && p.tern_int == 2 && d.np == 8) process_ternary_int8(e, d);
+      else process_ternary_int(e, d);
     } else if (fmt == KVC_FMT_TERNARY2) {
       constexpr int GB = HPC * group_bytes(KVC_FMT_TERNARY2, D);   // page stride
       e += wi * group_bytes(KVC_FMT_TERNARY2, D);
@@ -953,7 +1042,7 @@ struct Worker {
 
   // ------------------------------------------------------------- main
   __device__ __forceinline__ bool consume(int slot, uint32_t parity) {
-    if (!mbar_wait(&bars[slot], parity)) return false;
+    if (!mbar_wait(&bars[slot], parity, wait_limit)) return false;
     const Desc& d = desc[slot];
     const int bg = d.bg;
     if (bg != cur_bg) {
@@ -1003,6 +1092,11 @@ struct Worker {
     nxt_b_pending = true;
     nxa_pending = false;
 
+    // Failure-detection test mode: slot 0's first phase waits for 16 bytes
+    // that no copy delivers, so every wait on it runs out (after a few short
+    // tries) and the launch ends with the timeout flag.
+    wait_limit = p.test_timeout ? 4u : kSpinLimit;
+    if (p.test_timeout && wi == 0 && lane == 0) mbar_expect_tx(&bars[0], 16u);
     // warp 0 fills both slots first; later refills come from release()
     bool v0 = issue(0, wi == 0), v1 = issue(1, wi == 0);
     bool ok = true;
@@ -1016,8 +1110,8 @@ struct Worker {
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrTimeout);
       // let copies still in flight land before the CTA's memory is released
-      mbar_wait(&bars[0], 0u), mbar_wait(&bars[0], 1u);
-      mbar_wait(&bars[1], 0u), mbar_wait(&bars[1], 1u);
+      mbar_wait(&bars[0], 0u, wait_limit), mbar_wait(&bars[0], 1u, wait_limit);
+      mbar_wait(&bars[1], 0u, wait_limit), mbar_wait(&bars[1], 1u, wait_limit);
       return;
     }
     finish();

@@ -50,12 +50,29 @@ static bool umma_selected() {
 }
 
 // Ternary P.V of the tensor-core kernel at GQA <= 4: int8 MMAs with P in two
-// exact digits (default), or f16 MMAs with P as an f16 hi + lo pair when the
-// environment variable KVC_DECODE_TERNARY_PV is "f16" (read once per process).
-static bool ternary_pv_int() {
-  static const bool on = [] {
+// exact digits, full entries with one softmax maximum test per entry (2,
+// the default); the same per page pair (1, "pair"); or f16 MMAs with P as an
+// f16 hi + lo pair (0, "f16").  Environment variable KVC_DECODE_TERNARY_PV,
+// read once per process.
+static int ternary_pv_mode() {
+  static const int mode = [] {
     const char* v = getenv("KVC_DECODE_TERNARY_PV");
-    return v == nullptr || strcmp(v, "f16") != 0;
+    if (v != nullptr && strcmp(v, "f16") == 0) return 0;
+    if (v != nullptr && strcmp(v, "pair") == 0) return 1;
+    return 2;
+  }();
+  return mode;
+}
+
+// Failure-detection tests: with KVC_TEST_DECODE_TIMEOUT=1 (read once per
+// process) the tensor-core decode kernel arms its first ring slot for bytes
+// no copy delivers, so its bounded waits run out and it sets device flag 8
+// (read by kvc_decode_read_error); nothing faults or hangs, and the context
+// stays usable.
+static bool test_timeout() {
+  static const bool on = [] {
+    const char* v = getenv("KVC_TEST_DECODE_TIMEOUT");
+    return v != nullptr && strcmp(v, "1") == 0;
   }();
   return on;
 }
@@ -458,7 +475,8 @@ kvc_status kvc_decode_attention_paged_layers(const void* q_bf16, const kvc_paged
   p.hp = hp_mode;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.tern_int = kvc::ternary_pv_int() ? 1 : 0;
+  p.tern_int = kvc::ternary_pv_mode();
+  p.test_timeout = kvc::test_timeout() ? 1 : 0;
   p.n_splits = plan.n_splits;
   p.pages_per_split = plan.pages_per_split;
   p.out = out;

@@ -81,6 +81,8 @@ struct DecodeParams {
   int sink, window, hp;
   float scale_log2;          // softmax_scale * log2(e)
   int tern_int;              // tensor-core kernel, GQA <= 4: ternary P.V on int8 MMAs
+                             // (1: softmax per page pair; 2: per full entry), 0: f16
+  int test_timeout;          // tensor-core kernel: make the first slot wait run out (failure tests)
   int n_splits, pages_per_split;
   float* out;
   uint32_t* err;             // device error word

@@ -435,7 +435,13 @@ KVC_API kvc_status kvc_decode_plan_info(int batch, int n_q_heads, int n_kv_heads
  * running maximum, 2^-15 steps).  Environment, read once per process:
  * KVC_DECODE_KERNEL=tcgen05 selects the tensor-memory kernel;
  * KVC_DECODE_TERNARY_PV=f16 runs the ternary pages' P.V at GQA <= 4 on f16
- * MMAs (P as an f16 hi + lo pair) instead.
+ * MMAs (P as an f16 hi + lo pair) instead, =pair keeps the int8 products but
+ * tests the running maximum per page pair rather than once per full entry
+ * of 8 pages; KVC_TEST_DECODE_TIMEOUT=1 is a
+ * failure-detection test mode of the tensor-core kernel: its first ring
+ * slot waits for bytes no copy delivers, every bounded wait on it gives up
+ * after a few short tries, and the call sets flag 8 (output rows not
+ * written) without faulting or hanging.
  */
 KVC_API kvc_status kvc_decode_attention_paged(const void* q_bf16, const kvc_paged_cache* cache,
                                       const int32_t* block_table, const uint8_t* older_fmt,
