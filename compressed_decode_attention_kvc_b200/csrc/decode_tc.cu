@@ -616,9 +616,13 @@ struct Worker {
   // Threads with tig >= 2 read (and order) 2tig + 1, 2tig + 9, 2tig, 2tig + 8
   // instead, so that no two lanes of a load share a bank; their P digits are
   // swapped to match (pv_digits).
+  static constexpr int kVW4 = kBB < 4 ? 1 : kBB / 4;   // words of a V row this thread reads
   __device__ __forceinline__ void v_rows_t(const unsigned char* vg, uint32_t (&T)[kBB < 4 ? 4 : kBB]) {
-    constexpr int NW = kBB < 4 ? 1 : kBB / 4;
-    uint32_t r[4][NW];
+    uint32_t r[4][kVW4];
+    v_rows_ld(vg, r);
+    v_rows_tr(r, T);
+  }
+  __device__ __forceinline__ void v_rows_ld(const unsigned char* vg, uint32_t (&r)[4][kVW4]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int tok = 2 * tig + ((q & 1) ? 8 : 0) + ((q >> 1) ^ (tig >> 1));
@@ -633,8 +637,10 @@ struct Worker {
         r[q][1] = v.y;
       }
     }
+  }
+  __device__ __forceinline__ void v_rows_tr(const uint32_t (&r)[4][kVW4], uint32_t (&T)[kBB < 4 ? 4 : kBB]) {
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
+    for (int w = 0; w < kVW4; ++w) {
       const uint32_t x01 = prmt(r[0][w], r[1][w], 0x5140u), x23 = prmt(r[0][w], r[1][w], 0x7362u);
       const uint32_t y01 = prmt(r[2][w], r[3][w], 0x5140u), y23 = prmt(r[2][w], r[3][w], 0x7362u);
       T[4 * w + 0] = prmt(x01, y01, 0x5410u);
@@ -785,6 +791,11 @@ struct Worker {
     // only the entry's last page can be partial
     if (gid >= d.nrows) x[7][0] = -INFINITY;
     if (gid + 8 >= d.nrows) x[7][1] = -INFINITY;
+    // the first pair's V rows, loaded before the maximum test so that their
+    // latency overlaps it
+    uint32_t ra[4][kVW4], rb[4][kVW4];
+    v_rows_ld(e + S::kHalf, ra);
+    v_rows_ld(e + S::kHalf + GB, rb);
     float mx = x[0][0];
 #pragma unroll
     for (int pg = 0; pg < 8; ++pg) mx = fmaxf(mx, fmaxf(x[pg][0], x[pg][1]));
@@ -818,8 +829,13 @@ struct Worker {
     for (int pr2 = 0; pr2 < 4; ++pr2) {
       const int i = 2 * pr2;
       uint32_t TA[NT], TB[NT];
-      v_rows_t(e + S::kHalf + i * GB, TA);
-      v_rows_t(e + S::kHalf + (i + 1) * GB, TB);
+      if (pr2 == 0) {
+        v_rows_tr(ra, TA);
+        v_rows_tr(rb, TB);
+      } else {
+        v_rows_t(e + S::kHalf + i * GB, TA);
+        v_rows_t(e + S::kHalf + (i + 1) * GB, TB);
+      }
       const float p0 = ex2(x[i][0] - mm), p1 = ex2(x[i][1] - mm);
       const float p2 = ex2(x[i + 1][0] - mm), p3 = ex2(x[i + 1][1] - mm);
       l0 += (p0 + p1) + (p2 + p3);
