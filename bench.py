@@ -100,7 +100,7 @@ def load_peaks():
     if os.path.exists(path):
         d = json.load(open(path))
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
-    return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+    return 6650.0, "fallback (6.65 TB/s, an earlier copy-bandwidth measurement on B200)"
 
 
 # ---------------------------------------------------------------- bytes
