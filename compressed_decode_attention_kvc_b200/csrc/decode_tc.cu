@@ -8,35 +8,37 @@
 // "Core architecture" (codes {-1, 0, +1}, gamma = mean|X|, 4 codes per byte).
 //
 // Design (B200):
-// * Work: the (sequence, KV head, page) units of the whole batch are split
-//   over every warp of a persistent grid ("stream-K"), weighted by the bytes
-//   each page moves (a BF16 page of the window costs 8 ternary pages): warp
-//   W owns the units whose weighted start lies in [W*C/NW, (W+1)*C/NW), a
-//   range that may span several (sequence, KV head) pairs.  Each warp is an
-//   independent worker; no CTA-wide synchronisation after the prologue.
-//   Ragged context lengths and format mixes balance by construction.
-// * Staging: each warp keeps a 2-entry ring in shared memory; an 8 KB entry
-//   (4 KB at head_dim 64) holds the K groups then the V groups of up to 8
-//   ternary pages, 2 FP8 pages or one BF16 page (half a page at head_dim
-//   256) of one KV head, filled with 1-D TMA bulk copies (cp.async.bulk, no
-//   multicast) that complete on an mbarrier.  Page metadata (format, block-
-//   table slot, scales) for 32 units at a time is loaded lane-parallel one
-//   chunk ahead, so the warp never waits on a dependent global load.
-// * Math: mma.sync m16n8k16 (f16 in, f32 accumulate) with swapped operands:
-//   page tokens on M, the GQA group (<= 8 query heads) on N.  Q.K^T has the
-//   unpacked K page as A and Q as B; P.V has V^T as A and P^T as B (the
-//   score tile is transposed in registers with movmatrix).  Ternary codes are
-//   turned into f16 operands with one shift and one AND per pair of codes:
-//   the 2-bit field 01 / 11 placed at bits 14..15 of a half is +2.0 / -2.0
-//   exactly, 00 is 0.  FP8 pages convert with cvt.f16x2.e4m3x2, BF16 pages
-//   with a byte permute and cvt.f16x2.f32.  Tensor-core operands come from
-//   registers, so no unpacked copy of a page ever touches shared memory.
-// * Softmax: online, per page, in log2 units, with a lazy maximum: the
-//   running maximum moves (and the accumulators are rescaled) only when a
-//   score exceeds it by more than 2^8, so P stays within f16 range without a
-//   cross-lane max on every page.  Per-page V scales are folded into P relative to a
-//   per-warp reference scale that is re-based when the ratio leaves
-//   [1/16, 16], keeping P far from the f16 subnormal range.
+// * Work: the (sequence, KV-head group, page) units of the whole batch are
+//   split over the CTAs of a persistent grid ("stream-K"), weighted by the
+//   time a page costs: CTA W owns the units whose weighted start lies in
+//   [W*C/NW, (W+1)*C/NW), a range that may span several (sequence, head
+//   group) pairs, so ragged lengths and format mixes balance by
+//   construction.  A CTA has one warp per KV head of its group (4, 2 or 1);
+//   all its warps walk the same pages, each for its own head.
+// * Staging: each CTA keeps a 2-slot ring in shared memory (8 KB per head
+//   and slot; 4 KB at head_dim 64, 7 KB for two-head CTAs at head_dim 128),
+//   holding the K groups then the V groups of up to 8 ternary pages, FP8
+//   pages or one BF16 page (half a page where a slot is smaller), filled by
+//   1-D TMA bulk copies (cp.async.bulk, no multicast) that complete on an
+//   mbarrier; the heads' groups of a page are contiguous, so one copy moves
+//   a page for all of them.  Page metadata (format, block-table slot, scales)
+//   for 32 units at a time is loaded lane-parallel one chunk ahead.  The last
+//   warp to release a slot refills it.
+// * Math, register-sourced mma.sync, page tokens on M and the GQA group on N:
+//   Q.K^T of ternary pages on int8 MMAs (codes as +-64 bytes: one AND and
+//   one shift per four codes; Q as 15-bit int8 hi/lo digits per query head),
+//   of FP8 pages on f16 MMAs, of BF16 pages on bf16 MMAs.  P.V has V^T as A
+//   and P^T as B: with at most 4 query heads, ternary pages take one int8
+//   MMA per m-tile and page pair (P as two exact unsigned digits, int32 sums
+//   folded into fp32 once per entry); otherwise f16 / bf16 MMAs with P as a
+//   hi + lo pair (movmatrix transposes the score tile).  No unpacked copy of
+//   a page touches shared memory.
+// * Softmax: online, in log2 units.  Full entries of 8 ternary pages test
+//   the running maximum once (digit sums rescale exactly by shifts, since
+//   the maximum moves in whole log2 units) and run their P.V as one
+//   straight run of code; other entries use a lazy maximum that moves only
+//   when a score exceeds it by 2^8.  Per-page V scales are folded into P
+//   relative to a per-warp reference scale.
 // * Merge: each warp writes one partial state per (sequence, KV head) it
 //   touched; the last writer for a pair (an atomic ticket, no waiting)
 //   merges the pair's partials and writes the output rows.
