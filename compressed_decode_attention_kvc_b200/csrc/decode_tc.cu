@@ -34,10 +34,11 @@
 //   hi + lo pair (movmatrix transposes the score tile).  No unpacked copy of
 //   a page touches shared memory.
 // * Softmax: online, in log2 units.  Full entries of 8 ternary pages test
-//   the running maximum once (digit sums rescale exactly by shifts, since
-//   the maximum moves in whole log2 units) and run their P.V as one
-//   straight run of code; other entries use a lazy maximum that moves only
-//   when a score exceeds it by 2^8.  Per-page V scales are folded into P
+//   the running maximum once, take P's digits relative to the entry's own
+//   maximum and run their P.V as one straight run of code; shorter ternary
+//   entries at GQA <= 4 test it per page pair (the maximum moves in whole
+//   log2 units, so the digit sums rescale exactly by shifts); the other
+//   paths use a lazy maximum that moves only when a score exceeds it by 2^8.  Per-page V scales are folded into P
 //   relative to a per-warp reference scale.
 // * Merge: each warp writes one partial state per (sequence, KV head) it
 //   touched; the last writer for a pair (an atomic ticket, no waiting)
@@ -769,7 +770,8 @@ struct Worker {
   // 128): the scores of all 8 pages first, one test of the running maximum
   // for the whole entry, then the four page pairs' P.V as one straight run
   // of code, so the loads, transposes and MMAs of one pair overlap the
-  // softmax of the next.  Same arithmetic as process_ternary_int.
+  // softmax of the next.  P's digits are taken relative to the entry's own
+  // maximum (process_ternary_int: relative to the running maximum).
   __device__ __forceinline__ void process_ternary_int8(const unsigned char* e, const Desc& d) {
     constexpr int GB = HPC * group_bytes(KVC_FMT_TERNARY2, D);   // page stride
     constexpr int NT = kBB < 4 ? 4 : kBB;
@@ -825,7 +827,15 @@ struct Worker {
         }
       }
     }
-    const float mm = m0 == -INFINITY ? 0.f : m0;
+    // P's digits are taken relative to this entry's own maximum per head, so
+    // every entry keeps 15 bits of its largest P whatever the running
+    // maximum; sblk = 2^(entry maximum - m0) <= 1 scales the entry into the
+    // running state (the normaliser and the fold)
+    float rh = mx;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) rh = fmaxf(rh, __shfl_xor_sync(kFull, rh, o));
+    const float mm = rh == -INFINITY ? 0.f : rh;
+    const float sblk = (rh == -INFINITY || m0 == -INFINITY) ? 0.f : ex2(rh - m0);
     const uint32_t sw = tig >= 2 ? 0x1032u : 0x3210u;
 #pragma unroll
     for (int pr2 = 0; pr2 < 4; ++pr2) {
@@ -840,7 +850,7 @@ struct Worker {
       }
       const float p0 = ex2(x[i][0] - mm), p1 = ex2(x[i][1] - mm);
       const float p2 = ex2(x[i + 1][0] - mm), p3 = ex2(x[i + 1][1] - mm);
-      l0 += (p0 + p1) + (p2 + p3);
+      l0 += ((p0 + p1) + (p2 + p3)) * sblk;
       const float rA = d.vs[i] * r15, rB = d.vs[i + 1] * r15;
       const uint32_t f0 = __float_as_uint(fmaf(p0, rA, kMagic)), f1 = __float_as_uint(fmaf(p1, rA, kMagic));
       const uint32_t f2 = __float_as_uint(fmaf(p2, rB, kMagic)), f3 = __float_as_uint(fmaf(p3, rB, kMagic));
@@ -854,7 +864,7 @@ struct Worker {
         imma16832_su(ai[mt], tern8(TA[blo], f), tern8(TA[bhi], f), tern8(TB[blo], f), tern8(TB[bhi], f), b0, b1);
       }
     }
-    const float cf = gmax * (1.f / 2097152.f) * inv_uref;
+    const float cf = gmax * (1.f / 2097152.f) * inv_uref * sblk;
 #pragma unroll
     for (int mt = 0; mt < S::kSteps; ++mt) {
       acc[mt][0] += (float)(ai[mt][0] * 256 + ai[mt][1]) * cf;
